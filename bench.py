@@ -1,0 +1,374 @@
+#!/usr/bin/env python3
+"""Throughput of transposable N:M mask generation on B200 GPUs.
+
+One step = one call of the public entry point tsenor_mask over one whole
+synthetic weight matrix (Dykstra plan, sort, greedy, repair, local search,
+bit packing).  Default workload: 4096 x 11008 bf16, Student-t(3) x 0.02 with
+1% outlier columns x10, transposable 16:32, tau = 20, T = 300, L = 8.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank solves its own matrix of the same shape (a
+different seed): blocks are independent, so there is no data-path
+collective and the run scales weakly.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "w4096x11008_bf16_t3_16of32"
+SM_COUNT = 148
+MUFU_PER_CLK_PER_SM = 16          # ex2 / lg2 / rcp results per clock per SM
+SM_MAX_MHZ_FALLBACK = 1965.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=60)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    p.add_argument("--cpu-seconds", type=float, default=15.0,
+                   help="target CPU time of the bounded oracle sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args(argv)
+
+
+# --------------------------------------------------------------------------- helpers
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except OSError:
+        return {}
+
+
+def mufu_peak_tops(sm_mhz):
+    return SM_COUNT * MUFU_PER_CLK_PER_SM * sm_mhz * 1e6 / 1e12
+
+
+def source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_mask_search_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_key):
+    """DRAM bytes per launch from a committed ncu summary, if taken on today's sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel_key)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_digest") != source_digest():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        self.t0 = self.t1 = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            rows.append((ts, parts))
+        inside = [p for ts, p in rows if self.t0 is not None and self.t0 - 0.05 <= ts <= self.t1 + 0.05]
+        use = inside or [p for _, p in rows]
+        mhz = [float(p[1]) for p in use if p[1].replace(".", "").isdigit()]
+        mx = [float(p[2]) for p in use if p[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for p in use for k in range(4) if p[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(use), "samples_in_timed_region": len(inside),
+                "power_w_max": max((float(p[3]) for p in use if p[3].replace(".", "").isdigit()), default=None)}
+
+
+def to_device(storage, dtype, device):
+    import torch
+    if dtype == "bf16":
+        return torch.from_numpy(storage.view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(storage).to(device)
+
+
+# --------------------------------------------------------------------------- CPU (oracle) legs
+
+def oracle_sample(vals, w, seconds, cores=0):
+    """Oracle on the first k block-rows of the matrix, k sized for ~`seconds` of CPU work."""
+    import oracle
+    M = w.M
+    nbr = w.rows // M
+    t = time.perf_counter()
+    oracle.mask(vals[:M], w.N, M, w.tau, w.iters, w.sweeps, threads=cores)
+    t1 = max(time.perf_counter() - t, 1e-3)
+    k = int(max(1, min(nbr, seconds / t1)))
+    sub = np.ascontiguousarray(vals[:k * M])
+    t = time.perf_counter()
+    m_ref, _, st = oracle.mask(sub, w.N, M, w.tau, w.iters, w.sweeps, threads=cores)
+    dt = time.perf_counter() - t
+    return sub, k, dt, m_ref, st
+
+
+def cpu_baseline_leg(vals, w, gpu_mask_words, seconds):
+    """Oracle timing on a bounded sample, plus the gap of the GPU masks to the exact optimum there."""
+    import oracle
+    cores = oracle.threads_used(0)
+    sub, k, dt, m_ref, st = oracle_sample(vals, w, seconds)
+    params = sub.shape[0] * sub.shape[1]
+    opt, _ = oracle.opt(sub, w.N, w.M)
+    obj_gpu = oracle.objective(sub, gpu_mask_words[:sub.shape[0]], w.N, w.M)
+    obj_ref = oracle.objective(sub, m_ref, w.N, w.M)
+    gap = (opt - obj_gpu) / opt
+    gap_ref = (opt - obj_ref) / opt
+    pruned = (np.abs(sub).astype(np.float64).reshape(-1).sum() / opt.size)
+    return {
+        "cpu_baseline": {"value": params / dt / 1e9, "unit": "Gparams/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first {k} of {w.rows // w.M} block-rows ({k * (w.cols // w.M)} blocks, "
+                                   f"{params} params) of the same matrix; plain C, OpenMP over blocks",
+                         "seconds": dt},
+        "gap": {"mean": float(np.mean(gap)), "max": float(np.max(gap)),
+                "mean_vs_pruned_mass": float(np.mean((opt - obj_gpu) / np.maximum(pruned - opt, 1e-30))),
+                "oracle_mean": float(np.mean(gap_ref)), "blocks": int(opt.size),
+                "definition": "(opt - kept)/opt per block, opt = exact min-cost-flow optimum",
+                "pages_claim": "1-10% of optimal"},
+    }
+
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, on the host cores, on bounded samples of the workload."""
+    if rank != 0:
+        return
+    import oracle
+    w = synth.WORKLOADS[args.workload]
+    _, vals = synth.workload_matrix(w)
+    cores = oracle.threads_used(0)
+    M = w.M
+    t = time.perf_counter()
+    oracle.mask(vals[:M], w.N, M, w.tau, w.iters, w.sweeps)
+    t1 = max(time.perf_counter() - t, 1e-3)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    k = int(max(1, min(w.rows // M, budget / t1)))
+    sub = np.ascontiguousarray(vals[:k * M])
+    for _ in range(args.warmup):
+        oracle.mask(sub, w.N, M, w.tau, w.iters, w.sweeps)
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        oracle.mask(sub, w.N, M, w.tau, w.iters, w.sweeps)
+        times.append(time.perf_counter() - t)
+    params = sub.shape[0] * sub.shape[1]
+    step = statistics.mean(times)
+    value = params / step / 1e9
+    line = {"impl": "reference", "metric": "transposable N:M mask Gparams/s (oracle, host cores)",
+            "value": value, "unit": "Gparams/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "rows": w.rows, "cols": w.cols, "N": w.N, "M": w.M, "tau": w.tau,
+                       "iters": w.iters, "sweeps": w.sweeps, "sample_block_rows": k},
+            "cpu_baseline": {"value": value, "unit": "Gparams/s", "cores": cores, "kind": "oracle",
+                             "sample": f"first {k} block-rows ({params} params) per step"},
+            "e2e": {"value": value, "unit": "Gparams/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- GPU leg
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    import sparse_mask_search_b200 as tsl
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    w = synth.WORKLOADS[args.workload]
+    storage, vals = synth.workload_matrix(w, seed=w.seed + rank)
+    Wd = to_device(storage, w.dtype, dev)
+    wpr = (w.cols + 31) // 32
+    mask = torch.empty((w.rows, wpr), dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        tsl.tsenor_mask(Wd, w.N, w.M, w.tau, w.iters, w.sweeps, out=mask, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    time.sleep(0.3)
+
+    # ---- timed region: K steps, L2 flushed before each (outside the events)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.mark_start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        step()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.mark_end()
+    if world > 1:
+        dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    mean_ms = sum(step_ms) / len(step_ms)
+    t_max = torch.tensor([mean_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    mean_ms_max = float(t_max.item())
+    clocks = sampler.stop()
+    gpu_mask = mask.cpu().numpy().view(np.uint32)
+
+    # ---- dominant kernel alone (the Dykstra plan kernel), same stream, same input
+    plan = torch.empty((w.rows, w.cols), dtype=torch.float32, device=dev)
+    for _ in range(3):
+        tsl.tsenor_plan(Wd, w.N, w.M, w.tau, w.iters, out=plan, stream=stream)
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
+    for a, b in kev:
+        flush.zero_()
+        a.record(stream)
+        tsl.tsenor_plan(Wd, w.N, w.M, w.tau, w.iters, out=plan, stream=stream)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    plan_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    round_ms = max(mean_ms - plan_ms, 0.0)
+    del plan
+
+    # ---- end to end through the public API with host buffers
+    host_w = torch.from_numpy(storage.view(np.int16) if w.dtype == "bf16" else storage).pin_memory()
+    host_mask = torch.empty((w.rows, wpr), dtype=torch.int32).pin_memory()
+    W2 = torch.empty_like(Wd)
+    e2e_ev = []
+    n_e2e = max(3, min(args.steps, 20))
+    for k in range(n_e2e + 2):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.zero_()
+        a.record(stream)
+        W2.view(torch.int16 if w.dtype == "bf16" else torch.float32).copy_(host_w, non_blocking=True)
+        tsl.tsenor_mask(W2, w.N, w.M, w.tau, w.iters, w.sweeps, out=mask, stream=stream)
+        host_mask.copy_(mask, non_blocking=True)
+        b.record(stream)
+        if k >= 2:
+            e2e_ev.append((a, b))
+    torch.cuda.synchronize(dev)
+    e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in e2e_ev)
+    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_t.item())
+
+    params = w.rows * w.cols
+    value = params * world / (mean_ms_max / 1e3) / 1e9
+    ops_per_param = w.iters * (1.0 + 2.0 / w.M)
+    achieved = params * ops_per_param / (plan_ms / 1e3) / 1e12
+    peak = mufu_peak_tops(SM_MAX_MHZ_FALLBACK)
+    kernel_key = f"dykstra_tile_kernel<{w.M},{w.dtype}>" if w.M >= 16 else f"dykstra_thread_kernel<{w.M},{w.dtype}>"
+    traffic = profiled_traffic(kernel_key)
+    line = {
+        "metric": "transposable N:M mask Gparams/s at 1 B200 (% of roofline); mean gap to exact opt",
+        "value": value, "unit": "Gparams/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": mean_ms_max, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "rows": w.rows, "cols": w.cols, "input_dtype": w.dtype, "N": w.N,
+                   "M": w.M, "tau": w.tau, "iters": w.iters, "sweeps": w.sweeps,
+                   "l2": "flushed before every timed step (256 MiB memset outside the events)",
+                   "parallelism": f"replicas x{world}: each rank solves its own matrix, no collective"},
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TOP/s",
+                     "frac": achieved / peak, "traffic": traffic, "kernel": kernel_key,
+                     "ops": f"{ops_per_param:.2f} MUFU ops (ex2/lg2) per param = T*(1+2/M)",
+                     "peak_basis": f"{SM_COUNT} SMs x {MUFU_PER_CLK_PER_SM} MUFU/clk x {SM_MAX_MHZ_FALLBACK:.0f} MHz",
+                     "kernel_ms": plan_ms},
+        "breakdown_ms": {"plan_kernel": plan_ms, "rounding_and_rest": round_ms},
+        "e2e": {"value": params * world / (e2e_ms / 1e3) / 1e9, "unit": "Gparams/s",
+                "h2d_bytes_per_step": int(storage.nbytes), "d2h_bytes_per_step": int(host_mask.numel() * 4),
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": None,
+        "hbm": {"algorithmic_bytes_per_step": int(storage.nbytes + mask.numel() * 4),
+                "achieved_gbs": (storage.nbytes + mask.numel() * 4) / (mean_ms_max / 1e3) / 1e9,
+                "measured_peak_gbs": measured_peaks().get("hbm_gbs")},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line.update(cpu_baseline_leg(vals, w, gpu_mask, args.cpu_seconds))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

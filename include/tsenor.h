@@ -1,0 +1,127 @@
+/*
+ * tsenor.h -- C ABI of the B200 transposable N:M mask solver.
+ *
+ * The method is TSENOR, as described in "Pith review of TSENOR:
+ * Highly-Efficient Algorithm for Finding Transposable N:M Sparse Masks"
+ * (pith.science/paper/2505.23949):
+ *   - the problem ("Core claim"): split W into MxM blocks and, per block, find
+ *     a 0/1 mask with exactly N ones in every row and every column that
+ *     maximises the kept sum of |W|;
+ *   - the solver ("What carries the argument"): entropy-regularised
+ *     capacitated transport relaxation solved by Dykstra's alternating KL
+ *     projections in log space (row normalisation, column normalisation,
+ *     clip at 1 with a correction term), then rounding by a descending sort
+ *     with greedy row/column budgets, a feasibility repair and the
+ *     2-in/1-out swap local search;
+ *   - the free parameters ("Assumptions & free parameters"): tau, the
+ *     iteration count T and the local-search length L.
+ * The review prints no interface or code; this ABI is this library's own.
+ *
+ * Common conventions for every entry point:
+ *  - Pointers to W, the plan, the mask and the objective are DEVICE pointers
+ *    owned by the caller; the library keeps none of them after the call.
+ *    W and the plan must be 16-byte aligned; the mask 8-byte aligned.
+ *  - W is row-major, rows x cols, of the element type `dtype`; only |W| is
+ *    used.  rows and cols must be multiples of M (the review leaves other
+ *    shapes open, "Assumptions & free parameters"); rows == 0 or cols == 0
+ *    is a valid empty call that does nothing.
+ *  - Supported M: 4, 8, 16, 32, 64.  1 <= N <= M.  tau > 0 and finite,
+ *    iters >= 1, sweeps >= 0.
+ *  - The kernel of block b is x0_ij = tau * |W_ij| / max(|W| over b)
+ *    (x0 = 0 for an all-zero block); one iteration is a row step, a column
+ *    step and a clip.
+ *  - Mask layout: row-major, words_per_row = ceil(cols / 32) uint32 words
+ *    per row; bit k of word w of row r is column 32*w + k (least significant
+ *    bit first); bits past the last column are written as 0.
+ *  - All calls are asynchronous and ordered on `stream` (a cudaStream_t;
+ *    NULL is the legacy default stream).  Argument errors are detected on
+ *    the host before anything is enqueued and return at once.
+ *  - A block whose W holds NaN or Inf gets an all-zero mask and bumps the
+ *    device failure counter read by tsenor_error_count; the other blocks of
+ *    the call are unaffected.
+ *  - The library is not re-entrant across host threads for the same device
+ *    failure counter: concurrent calls add into one counter.
+ */
+#ifndef TSENOR_H
+#define TSENOR_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* tsenor_stream_t;   /* same type as cudaStream_t */
+
+typedef enum { TSENOR_F32 = 0, TSENOR_BF16 = 1 } tsenor_dtype;
+
+typedef enum {
+    TSENOR_OK = 0,
+    TSENOR_ERR_ARG = -1,             /* null pointer, bad dtype, N/tau/iters/sweeps out of range, misaligned pointer */
+    TSENOR_ERR_SHAPE = -2,           /* rows or cols negative or not a multiple of M */
+    TSENOR_ERR_UNSUPPORTED_M = -3,   /* M not in {4, 8, 16, 32, 64} */
+    TSENOR_ERR_CUDA = -4             /* a CUDA runtime call failed; see tsenor_last_error() */
+} tsenor_status;
+
+/*
+ * Transposable N:M mask of W (the whole hot path: Dykstra plan, sort, greedy,
+ * repair, local search, bit packing).
+ *   mask_out: rows x words_per_row uint32, written completely.
+ *   sweeps:   local-search sweeps L; one sweep visits every anchor row once.
+ * Uses a stream-ordered workspace of rows*cols floats (cudaMallocAsync /
+ * cudaFreeAsync on `stream`) that holds the plan between its two kernels.
+ */
+tsenor_status tsenor_mask(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
+                          int N, int M, float tau, int iters, int sweeps,
+                          uint32_t* mask_out, tsenor_stream_t stream);
+
+/*
+ * The fractional transport plan only: S = exp(x) after the clip of the last
+ * Dykstra iteration ("What carries the argument"), fp32, rows x cols,
+ * row-major, every block at its place in W.  0 <= S <= 1.  A block with
+ * non-finite W gets NaN.
+ */
+tsenor_status tsenor_plan(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
+                          int N, int M, float tau, int iters, float* plan_out,
+                          tsenor_stream_t stream);
+
+/*
+ * The rounding only, from a given plan (keys): per block, sort entries by
+ * (plan desc, |W| desc, flat index i*M+j asc), greedy with row/column
+ * budgets N, feasibility repair by 2-in/1-out moves, then `sweeps` sweeps of
+ * the swap local search, then bit packing into mask_out.
+ * plan: rows x cols fp32 (non-negative; a block holding NaN fails).
+ */
+tsenor_status tsenor_round(const float* plan, const void* W, tsenor_dtype dtype,
+                           int64_t rows, int64_t cols, int N, int M, int sweeps,
+                           uint32_t* mask_out, tsenor_stream_t stream);
+
+/*
+ * Kept mass per block: out[b] = sum over block b of |W_ij| * mask_ij in fp64,
+ * or NaN when a row or a column of block b does not hold exactly N ones.
+ * Blocks are numbered row-major over the block grid: b = (r/M)*(cols/M) + c/M.
+ *   out: (rows/M)*(cols/M) doubles (device).
+ */
+tsenor_status tsenor_objective(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
+                               const uint32_t* mask, int N, int M, double* out,
+                               tsenor_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns in *count_out the number of blocks that
+ * failed on this device (non-finite input, or a rounding step that found no
+ * move) since the previous call, and resets the counter.
+ */
+tsenor_status tsenor_error_count(tsenor_stream_t stream, int64_t* count_out);
+
+/* Static description of a status code. */
+const char* tsenor_status_string(int status);
+
+/* Message of the last TSENOR_ERR_CUDA on the calling host thread ("" if none). */
+const char* tsenor_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TSENOR_H */

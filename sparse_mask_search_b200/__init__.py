@@ -1,0 +1,146 @@
+"""Python binding of the B200 transposable N:M mask library (include/tsenor.h).
+
+Argument marshalling only: every step of the solver runs in the CUDA kernels
+of libtsenor_b200.so.  PyTorch provides device memory and streams.  There is
+no CPU fallback: if the library is missing, importing a function raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libtsenor_b200.so")
+
+TSENOR_F32, TSENOR_BF16 = 0, 1
+STATUS = {0: "TSENOR_OK", -1: "TSENOR_ERR_ARG", -2: "TSENOR_ERR_SHAPE", -3: "TSENOR_ERR_UNSUPPORTED_M",
+          -4: "TSENOR_ERR_CUDA"}
+EXPORTS = ("tsenor_mask", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
+           "tsenor_status_string", "tsenor_last_error")
+
+_lib = None
+
+
+class TsenorError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def lib() -> C.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m sparse_mask_search_b200.build` (nvcc, sm_100a)")
+        L = C.CDLL(LIB_PATH)
+        p, i64, i32, f32 = C.c_void_p, C.c_int64, C.c_int, C.c_float
+        L.tsenor_mask.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p]
+        L.tsenor_plan.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, p, p]
+        L.tsenor_round.argtypes = [p, p, i32, i64, i64, i32, i32, i32, p, p]
+        L.tsenor_objective.argtypes = [p, i32, i64, i64, p, i32, i32, p, p]
+        L.tsenor_error_count.argtypes = [p, C.POINTER(C.c_int64)]
+        L.tsenor_status_string.argtypes = [i32]
+        L.tsenor_status_string.restype = C.c_char_p
+        L.tsenor_last_error.restype = C.c_char_p
+        for name in EXPORTS:
+            getattr(L, name).restype = getattr(L, name).restype or C.c_int
+        _lib = L
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        L = lib()
+        msg = L.tsenor_status_string(status).decode()
+        if status == -4:
+            msg += ": " + L.tsenor_last_error().decode()
+        raise TsenorError(status, msg)
+
+
+def _stream_handle(stream) -> int | None:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(W) -> int:
+    import torch
+    if W.dtype == torch.bfloat16:
+        return TSENOR_BF16
+    if W.dtype == torch.float32:
+        return TSENOR_F32
+    raise TypeError(f"W must be bfloat16 or float32, got {W.dtype}")
+
+
+def words_per_row(cols: int) -> int:
+    return (cols + 31) // 32
+
+
+def _check_2d_cuda(t, name):
+    if not t.is_cuda or t.dim() != 2 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous 2-D CUDA tensor")
+
+
+def tsenor_mask(W, N: int, M: int, tau: float, iters: int, sweeps: int, out=None, stream=None):
+    """Transposable N:M mask of W; returns (rows, ceil(cols/32)) int32 words (bit patterns)."""
+    import torch
+    _check_2d_cuda(W, "W")
+    rows, cols = W.shape
+    if out is None:
+        out = torch.empty((rows, words_per_row(cols)), dtype=torch.int32, device=W.device)
+    _check(lib().tsenor_mask(W.data_ptr(), _dtype_code(W), rows, cols, N, M, float(tau), iters, sweeps,
+                             out.data_ptr(), _stream_handle(stream)))
+    return out
+
+
+def tsenor_plan(W, N: int, M: int, tau: float, iters: int, out=None, stream=None):
+    """Fractional plan S (fp32, same shape as W) after `iters` Dykstra iterations."""
+    import torch
+    _check_2d_cuda(W, "W")
+    rows, cols = W.shape
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.float32, device=W.device)
+    _check(lib().tsenor_plan(W.data_ptr(), _dtype_code(W), rows, cols, N, M, float(tau), iters,
+                             out.data_ptr(), _stream_handle(stream)))
+    return out
+
+
+def tsenor_round(plan, W, N: int, M: int, sweeps: int, out=None, stream=None):
+    """Rounding of a given fp32 plan into a mask (int32 words)."""
+    import torch
+    _check_2d_cuda(W, "W")
+    _check_2d_cuda(plan, "plan")
+    rows, cols = W.shape
+    if plan.shape != W.shape or plan.dtype != torch.float32:
+        raise ValueError("plan must be float32 with the shape of W")
+    if out is None:
+        out = torch.empty((rows, words_per_row(cols)), dtype=torch.int32, device=W.device)
+    _check(lib().tsenor_round(plan.data_ptr(), W.data_ptr(), _dtype_code(W), rows, cols, N, M, sweeps,
+                              out.data_ptr(), _stream_handle(stream)))
+    return out
+
+
+def tsenor_objective(W, mask, N: int, M: int, out=None, stream=None):
+    """Per-block kept sum of |W| (fp64), NaN where a block row/column is not N:M."""
+    import torch
+    _check_2d_cuda(W, "W")
+    rows, cols = W.shape
+    if out is None:
+        out = torch.empty(((rows // M) * (cols // M),), dtype=torch.float64, device=W.device)
+    _check(lib().tsenor_objective(W.data_ptr(), _dtype_code(W), rows, cols, mask.data_ptr(), N, M,
+                                  out.data_ptr(), _stream_handle(stream)))
+    return out
+
+
+def tsenor_error_count(stream=None) -> int:
+    """Blocks that failed since the previous call (synchronises the stream)."""
+    n = C.c_int64(0)
+    _check(lib().tsenor_error_count(_stream_handle(stream), C.byref(n)))
+    return int(n.value)
+
+
+__all__ = ["tsenor_mask", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
+           "TsenorError", "lib", "words_per_row", "EXPORTS", "LIB_PATH"]

@@ -1,0 +1,356 @@
+// Dykstra's algorithm for the entropic capacitated transport relaxation of
+// every MxM block ("What carries the argument" and "Core claim" of the TSENOR
+// review; minor comment 2 on Algorithm 1).
+//
+// Math used by every kernel here (exact in real arithmetic):
+//  * State in base-2 log units.  After a clip, x = min(y, 0) and the Dykstra
+//    correction is logQ = max(y, 0) for y = x + logQ, so one number y per
+//    entry carries both.  Starting from y0 = (x0 - tau) * log2(e) keeps
+//    y0 <= 0 (so logQ0 = 0) and changes nothing: the first row step is blind
+//    to a constant shift of a row.
+//  * One iteration with e_ij = 2^min(y_ij, 0):
+//        R_i = sum_j e_ij          r_i = log2 N - log2 R_i     (row step)
+//        C_j = sum_i e_ij N / R_i  c_j = log2 N - log2 C_j     (column step,
+//                                  reusing the row step's exponentials)
+//        y_ij += r_i + c_j                                     (clip folded in)
+//    so one exponential per entry and iteration, plus one log per row and
+//    one per column.
+//  * The plan is S = 2^min(y, 0) after the last iteration; S = 1 exactly
+//    for clipped entries (y >= 0).
+#pragma once
+
+#include "common.cuh"
+
+namespace tsenor {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// M = 4, 8: one thread holds a whole block in registers.  Rows are streamed:
+// the exponentials of one row live only until its column contributions are
+// added, so no cross-thread traffic is needed at all.
+// ---------------------------------------------------------------------------
+template <int M, typename T>
+__global__ void __launch_bounds__(128)
+dykstra_thread_kernel(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks,
+                      int N, float tau, int iters, float* __restrict__ plan) {
+    const int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (b >= n_blocks) return;
+    const int64_t nbc = cols / M;
+    const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
+
+    float y[M][M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+        const typename T::storage* src = W + (r0 + i) * cols + c0;
+        if constexpr (M * sizeof(typename T::storage) >= 16) {
+#pragma unroll
+            for (int v = 0; v < M / T::kVec; ++v) T::load16(src + v * T::kVec, &y[i][v * T::kVec]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < M; ++j) y[i][j] = T::load1(src + j);
+        }
+    }
+    float m = 0.f;
+    bool finite = true;
+#pragma unroll
+    for (int i = 0; i < M; ++i)
+#pragma unroll
+        for (int j = 0; j < M; ++j) {
+            finite = finite && (y[i][j] <= 3.402823466e38f);   // false for NaN and Inf
+            m = fmaxf(m, y[i][j]);
+        }
+    const float tau2 = tau * kLog2e;
+#pragma unroll
+    for (int i = 0; i < M; ++i)
+#pragma unroll
+        for (int j = 0; j < M; ++j) {
+            const float q = m > 0.f ? __fdiv_rn(y[i][j], m) : 0.f;
+            y[i][j] = fmaf(tau2, q, -tau2);
+        }
+    const float fN = float(N), log2N = log2f(float(N));
+
+    if (finite) {
+        for (int t = 0; t < iters; ++t) {
+            float C[M];
+#pragma unroll
+            for (int j = 0; j < M; ++j) C[j] = 0.f;
+#pragma unroll
+            for (int i = 0; i < M; ++i) {
+                float e[M], R = 0.f;
+#pragma unroll
+                for (int j = 0; j < M; ++j) {
+                    e[j] = ex2(fminf(y[i][j], 0.f));
+                    R += e[j];
+                }
+                const float w = fN * rcp(R);
+                const float r = log2N - lg2(R);
+#pragma unroll
+                for (int j = 0; j < M; ++j) {
+                    C[j] = fmaf(e[j], w, C[j]);
+                    y[i][j] += r;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < M; ++j) {
+                const float c = log2N - lg2(C[j]);
+#pragma unroll
+                for (int i = 0; i < M; ++i) y[i][j] += c;
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+        float s[M];
+#pragma unroll
+        for (int j = 0; j < M; ++j)
+            s[j] = !finite ? __int_as_float(0x7fc00000) : (y[i][j] >= 0.f ? 1.f : ex2(y[i][j]));
+        float* dst = plan + (r0 + i) * cols + c0;
+#pragma unroll
+        for (int v = 0; v < M / 4; ++v)
+            reinterpret_cast<float4*>(dst)[v] = make_float4(s[4 * v], s[4 * v + 1], s[4 * v + 2], s[4 * v + 3]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// M = 16, 32, 64: a block is spread over M*M/32 threads, each holding a
+// P x Q = 4 x 8 sub-tile.  Threads of one block: t = rg * CG + cg with
+// cg in [0, CG = M/8) (lowest lane bits: the threads that share rows) and
+// rg in [0, RG = M/4) (the threads that share columns).
+//
+// Row and column sums are formed by a shuffle reduce-scatter in which every
+// thread keeps its registers in an order permuted by XOR with its own group
+// index; with that order every level of the butterfly sends the upper half
+// of the live registers to the partner and keeps the lower half, with no
+// lane-dependent selects.  The matching all-gather returns the row and
+// column potentials in the same permuted order.
+// ---------------------------------------------------------------------------
+template <int M>
+struct TileCfg {
+    static constexpr int P = 4, Q = 8;
+    static constexpr int CG = M / Q;                 // threads sharing a row
+    static constexpr int RG = M / P;                 // threads sharing a column
+    static constexpr int TPB = CG * RG;              // threads per block
+    static constexpr int BPW = TPB < 32 ? 32 / TPB : 1;   // blocks per warp
+    static constexpr int RSR = CG < P ? CG : P;      // lanes in the row reduce-scatter
+    static constexpr int ARR = CG / RSR;             // lanes in the row all-reduce after it
+    static constexpr int RO = P / RSR;               // rows owned per thread
+    static constexpr int CW = (RG < 32 / CG) ? RG : 32 / CG;   // column sharers inside a warp
+    static constexpr int RSC = CW < Q ? CW : Q;      // lanes in the column reduce-scatter
+    static constexpr int CO = Q / RSC;               // columns owned per thread
+    static constexpr int WC = RG / CW;               // warps sharing a column
+    static constexpr int THREADS = 128;              // CTA size
+    static constexpr int BPC = THREADS / TPB;        // blocks per CTA
+    static_assert(P * Q == 32, "sub-tile of 32 entries");
+    static_assert(TPB <= THREADS, "block larger than a CTA");
+    static_assert(CG * RSC == 32 || WC == 1, "cross-warp columns need full warps");
+};
+
+template <int M, typename T>
+__global__ void __launch_bounds__(128)
+dykstra_tile_kernel(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks,
+                    int N, float tau, int iters, float* __restrict__ plan) {
+    using C = TileCfg<M>;
+    constexpr int P = C::P, Q = C::Q;
+    extern __shared__ float smem[];
+    // tile staging: one M x M float tile per block of the CTA
+    float* tiles = smem;
+    float* colbuf = smem + C::BPC * M * M;   // [2][warps][32][CO] for cross-warp columns
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int blk = tid / C::TPB;                  // block slot within the CTA
+    const int t = tid % C::TPB;                    // thread within the block
+    const int cg = t % C::CG, rg = t / C::CG;
+    const int64_t b = int64_t(blockIdx.x) * C::BPC + blk;
+    const bool active = b < n_blocks;
+    const int64_t nbc = cols / M;
+    const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
+    float* tile = tiles + blk * M * M;
+
+    // ---- stage |W| of the block in shared memory (16-byte coalesced loads)
+    {
+        constexpr int V = T::kVec;
+        constexpr int CPR = M / V;                 // 16-byte chunks per tile row
+        for (int q = t; q < M * CPR; q += C::TPB) {
+            const int i = q / CPR, v = q % CPR;
+            float tmp[V];
+            if (active) T::load16(W + (r0 + i) * cols + c0 + v * V, tmp);
+            else {
+#pragma unroll
+                for (int u = 0; u < V; ++u) tmp[u] = 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < V; ++u) tile[i * M + v * V + u] = tmp[u];
+        }
+    }
+    __syncthreads();
+
+    // permuted local row / column of register k / c
+    const int gr = cg % C::RSR;                     // index in the row reduce-scatter group
+    const int gc = rg % C::RSC;                     // index in the column reduce-scatter group
+    auto lrow = [&](int k) { return ((k / C::RO) ^ gr) * C::RO + (k % C::RO); };
+    auto lcol = [&](int c) { return ((c / C::CO) ^ gc) * C::CO + (c % C::CO); };
+
+    float y[P][Q];
+    float m = 0.f;
+    bool finite = true;
+#pragma unroll
+    for (int k = 0; k < P; ++k)
+#pragma unroll
+        for (int c = 0; c < Q; ++c) {
+            const float a = tile[(P * rg + lrow(k)) * M + Q * cg + lcol(c)];
+            y[k][c] = a;
+            finite = finite && (a <= 3.402823466e38f);
+            m = fmaxf(m, a);
+        }
+    // block max and finiteness over the block's threads
+    if constexpr (C::TPB <= 32) {
+#pragma unroll
+        for (int s = 1; s < C::TPB; s <<= 1) {
+            m = fmaxf(m, __shfl_xor_sync(kFullMask, m, s));
+            finite = __shfl_xor_sync(kFullMask, int(finite), s) && finite;
+        }
+    } else {
+#pragma unroll
+        for (int s = 1; s < 32; s <<= 1) {
+            m = fmaxf(m, __shfl_xor_sync(kFullMask, m, s));
+            finite = __shfl_xor_sync(kFullMask, int(finite), s) && finite;
+        }
+        __shared__ float red_m[4];
+        __shared__ int red_f[4];
+        if (lane == 0) { red_m[warp] = m; red_f[warp] = finite; }
+        __syncthreads();
+        m = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
+        finite = red_f[0] && red_f[1] && red_f[2] && red_f[3];
+    }
+    const float tau2 = tau * kLog2e;
+#pragma unroll
+    for (int k = 0; k < P; ++k)
+#pragma unroll
+        for (int c = 0; c < Q; ++c) {
+            const float q = m > 0.f ? __fdiv_rn(y[k][c], m) : 0.f;
+            y[k][c] = fmaf(tau2, q, -tau2);
+        }
+    const float fN = float(N), log2N = log2f(float(N));
+
+    // Blocks of one warp (M = 16) may differ in finiteness; all lanes run the
+    // loop so that the shuffles stay converged, and a non-finite block's
+    // result is replaced by NaN at the end.
+    const bool run = (C::TPB <= 32) ? (__any_sync(kFullMask, finite) != 0) : finite;
+    if (run) {
+        for (int it = 0; it < iters; ++it) {
+            float e[P][Q];
+            float rs[P];
+#pragma unroll
+            for (int k = 0; k < P; ++k) {
+                rs[k] = 0.f;
+#pragma unroll
+                for (int c = 0; c < Q; ++c) {
+                    e[k][c] = ex2(fminf(y[k][c], 0.f));
+                    rs[k] += e[k][c];
+                }
+            }
+            // row reduce-scatter over RSR lanes, then all-reduce over ARR
+#pragma unroll
+            for (int s = C::RSR / 2; s >= 1; s >>= 1)
+#pragma unroll
+                for (int hi = 0; hi < s; ++hi)
+#pragma unroll
+                    for (int lo = 0; lo < C::RO; ++lo)
+                        rs[hi * C::RO + lo] += __shfl_xor_sync(kFullMask, rs[(hi + s) * C::RO + lo], s);
+#pragma unroll
+            for (int s = C::RSR; s < C::CG; s <<= 1)
+#pragma unroll
+                for (int lo = 0; lo < C::RO; ++lo)
+                    rs[lo] += __shfl_xor_sync(kFullMask, rs[lo], s);
+            // owned rows: scale w = N / R and log potential r = log2 N - log2 R
+            float wv[P], rv[P];
+#pragma unroll
+            for (int lo = 0; lo < C::RO; ++lo) {
+                wv[lo] = fN * rcp(rs[lo]);
+                rv[lo] = log2N - lg2(rs[lo]);
+            }
+            // all-gather back into the permuted register order
+#pragma unroll
+            for (int s = 1; s < C::RSR; s <<= 1)
+#pragma unroll
+                for (int hi = 0; hi < s; ++hi)
+#pragma unroll
+                    for (int lo = 0; lo < C::RO; ++lo) {
+                        wv[(hi + s) * C::RO + lo] = __shfl_xor_sync(kFullMask, wv[hi * C::RO + lo], s);
+                        rv[(hi + s) * C::RO + lo] = __shfl_xor_sync(kFullMask, rv[hi * C::RO + lo], s);
+                    }
+            // column partial sums of e * w
+            float cs[Q];
+#pragma unroll
+            for (int c = 0; c < Q; ++c) {
+                float acc = e[0][c] * wv[0];
+#pragma unroll
+                for (int k = 1; k < P; ++k) acc = fmaf(e[k][c], wv[k], acc);
+                cs[c] = acc;
+            }
+#pragma unroll
+            for (int s = C::RSC / 2; s >= 1; s >>= 1)
+#pragma unroll
+                for (int hi = 0; hi < s; ++hi)
+#pragma unroll
+                    for (int lo = 0; lo < C::CO; ++lo)
+                        cs[hi * C::CO + lo] += __shfl_xor_sync(kFullMask, cs[(hi + s) * C::CO + lo], s * C::CG);
+            if constexpr (C::WC > 1) {
+                float* buf = colbuf + (it & 1) * (4 * 32 * C::CO);
+#pragma unroll
+                for (int lo = 0; lo < C::CO; ++lo) buf[(warp * 32 + lane) * C::CO + lo] = cs[lo];
+                __syncthreads();
+#pragma unroll
+                for (int lo = 0; lo < C::CO; ++lo) {
+                    float acc = buf[(0 * 32 + lane) * C::CO + lo];
+#pragma unroll
+                    for (int w2 = 1; w2 < C::WC; ++w2) acc += buf[(w2 * 32 + lane) * C::CO + lo];
+                    cs[lo] = acc;
+                }
+            }
+            float cv[Q];
+#pragma unroll
+            for (int lo = 0; lo < C::CO; ++lo) cv[lo] = log2N - lg2(cs[lo]);
+#pragma unroll
+            for (int s = 1; s < C::RSC; s <<= 1)
+#pragma unroll
+                for (int hi = 0; hi < s; ++hi)
+#pragma unroll
+                    for (int lo = 0; lo < C::CO; ++lo)
+                        cv[(hi + s) * C::CO + lo] = __shfl_xor_sync(kFullMask, cv[hi * C::CO + lo], s * C::CG);
+#pragma unroll
+            for (int k = 0; k < P; ++k)
+#pragma unroll
+                for (int c = 0; c < Q; ++c) y[k][c] += rv[k] + cv[c];
+        }
+    }
+
+    // ---- plan S = 2^min(y,0) (1 exactly when clipped), via the smem tile
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < P; ++k)
+#pragma unroll
+        for (int c = 0; c < Q; ++c) {
+            const float s = !finite ? __int_as_float(0x7fc00000) : (y[k][c] >= 0.f ? 1.f : ex2(y[k][c]));
+            tile[(P * rg + lrow(k)) * M + Q * cg + lcol(c)] = s;
+        }
+    __syncthreads();
+    if (active) {
+        constexpr int CPR = M / 4;
+        for (int q = t; q < M * CPR; q += C::TPB) {
+            const int i = q / CPR, v = q % CPR;
+            const float4 val = *reinterpret_cast<const float4*>(tile + i * M + 4 * v);
+            *reinterpret_cast<float4*>(plan + (r0 + i) * cols + c0 + 4 * v) = val;
+        }
+    }
+}
+
+template <int M>
+constexpr size_t dykstra_tile_smem() {
+    using C = TileCfg<M>;
+    return sizeof(float) * (C::BPC * M * M + (C::WC > 1 ? 2 * 4 * 32 * C::CO : 0));
+}
+
+}  // namespace tsenor

@@ -1,0 +1,200 @@
+// Host side of the C ABI declared in include/tsenor.h: argument checks,
+// dispatch on M and dtype, stream-ordered launches, the failure counter.
+#include <cstdio>
+#include <cstring>
+#include <type_traits>
+
+#include "../../include/tsenor.h"
+#include "common.cuh"
+#include "dykstra.cuh"
+#include "rounding.cuh"
+#include "objective.cuh"
+
+namespace tsenor {
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+tsenor_status cuda_fail(cudaError_t e, const char* what) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, cudaGetErrorString(e));
+    return TSENOR_ERR_CUDA;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+tsenor_status check_common(const void* W, int dtype, int64_t rows, int64_t cols, int N, int M) {
+    if (M != 4 && M != 8 && M != 16 && M != 32 && M != 64) return TSENOR_ERR_UNSUPPORTED_M;
+    if (dtype != TSENOR_F32 && dtype != TSENOR_BF16) return TSENOR_ERR_ARG;
+    if (N < 1 || N > M) return TSENOR_ERR_ARG;
+    if (rows < 0 || cols < 0 || rows % M || cols % M) return TSENOR_ERR_SHAPE;
+    if (rows > (int64_t(1) << 31) || cols > (int64_t(1) << 31)) return TSENOR_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return TSENOR_OK;
+    if (!W || !aligned(W, 16)) return TSENOR_ERR_ARG;
+    return TSENOR_OK;
+}
+
+template <int M, typename T>
+cudaError_t launch_plan(const void* W, int64_t rows, int64_t cols, int N, float tau, int iters,
+                        float* plan, cudaStream_t st) {
+    const int64_t nb = (rows / M) * (cols / M);
+    const auto* w = static_cast<const typename T::storage*>(W);
+    if constexpr (M <= 8) {
+        const int64_t grid = (nb + 127) / 128;
+        dykstra_thread_kernel<M, T><<<dim3(unsigned(grid)), 128, 0, st>>>(w, cols, nb, N, tau, iters, plan);
+    } else {
+        constexpr size_t smem = dykstra_tile_smem<M>();
+        cudaError_t e = cudaFuncSetAttribute(dykstra_tile_kernel<M, T>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        const int64_t grid = (nb + TileCfg<M>::BPC - 1) / TileCfg<M>::BPC;
+        dykstra_tile_kernel<M, T><<<dim3(unsigned(grid)), TileCfg<M>::THREADS, smem, st>>>(
+            w, cols, nb, N, tau, iters, plan);
+    }
+    return cudaGetLastError();
+}
+
+template <int M, typename T>
+cudaError_t launch_round(const float* plan, const void* W, int64_t rows, int64_t cols, int N,
+                         int sweeps, uint32_t* mask, cudaStream_t st) {
+    const int64_t nb = (rows / M) * (cols / M);
+    const int64_t wpr = (cols + 31) / 32;
+    if (M == 4 || ((M == 8 || M == 16) && cols % 32)) {
+        // sub-word blocks: zero first so padding bits are 0 (and M = 4 can OR)
+        cudaError_t e = cudaMemsetAsync(mask, 0, size_t(rows) * size_t(wpr) * 4, st);
+        if (e != cudaSuccess) return e;
+    }
+    constexpr size_t smem = round_smem<M>();
+    cudaError_t e = cudaFuncSetAttribute(round_kernel<M, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(smem));
+    if (e != cudaSuccess) return e;
+    constexpr int WP = RoundCfg<M>::WARPS;
+    const int64_t grid = (nb + WP - 1) / WP;
+    round_kernel<M, T><<<dim3(unsigned(grid)), WP * 32, smem, st>>>(
+        plan, static_cast<const typename T::storage*>(W), cols, nb, N, sweeps, mask, wpr);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t dispatch_plan(int M, const void* W, int64_t rows, int64_t cols, int N, float tau, int iters,
+                          float* plan, cudaStream_t st) {
+    switch (M) {
+        case 4: return launch_plan<4, T>(W, rows, cols, N, tau, iters, plan, st);
+        case 8: return launch_plan<8, T>(W, rows, cols, N, tau, iters, plan, st);
+        case 16: return launch_plan<16, T>(W, rows, cols, N, tau, iters, plan, st);
+        case 32: return launch_plan<32, T>(W, rows, cols, N, tau, iters, plan, st);
+        default: return launch_plan<64, T>(W, rows, cols, N, tau, iters, plan, st);
+    }
+}
+
+template <typename T>
+cudaError_t dispatch_round(int M, const float* plan, const void* W, int64_t rows, int64_t cols, int N,
+                           int sweeps, uint32_t* mask, cudaStream_t st) {
+    switch (M) {
+        case 4: return launch_round<4, T>(plan, W, rows, cols, N, sweeps, mask, st);
+        case 8: return launch_round<8, T>(plan, W, rows, cols, N, sweeps, mask, st);
+        case 16: return launch_round<16, T>(plan, W, rows, cols, N, sweeps, mask, st);
+        case 32: return launch_round<32, T>(plan, W, rows, cols, N, sweeps, mask, st);
+        default: return launch_round<64, T>(plan, W, rows, cols, N, sweeps, mask, st);
+    }
+}
+
+cudaError_t run_plan(int dtype, int M, const void* W, int64_t rows, int64_t cols, int N, float tau,
+                     int iters, float* plan, cudaStream_t st) {
+    return dtype == TSENOR_BF16 ? dispatch_plan<BF16>(M, W, rows, cols, N, tau, iters, plan, st)
+                                : dispatch_plan<F32>(M, W, rows, cols, N, tau, iters, plan, st);
+}
+
+cudaError_t run_round(int dtype, int M, const float* plan, const void* W, int64_t rows, int64_t cols,
+                      int N, int sweeps, uint32_t* mask, cudaStream_t st) {
+    return dtype == TSENOR_BF16 ? dispatch_round<BF16>(M, plan, W, rows, cols, N, sweeps, mask, st)
+                                : dispatch_round<F32>(M, plan, W, rows, cols, N, sweeps, mask, st);
+}
+
+bool solver_params_ok(float tau, int iters) {
+    return tau > 0.f && tau <= 3.0e38f && iters >= 1;
+}
+
+}  // namespace
+}  // namespace tsenor
+
+using namespace tsenor;
+
+extern "C" tsenor_status tsenor_plan(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols, int N,
+                                     int M, float tau, int iters, float* plan_out, tsenor_stream_t stream) {
+    tsenor_status s = check_common(W, dtype, rows, cols, N, M);
+    if (s != TSENOR_OK) return s;
+    if (!solver_params_ok(tau, iters)) return TSENOR_ERR_ARG;
+    if (rows == 0 || cols == 0) return TSENOR_OK;
+    if (!plan_out || !aligned(plan_out, 16)) return TSENOR_ERR_ARG;
+    cudaError_t e = run_plan(dtype, M, W, rows, cols, N, tau, iters, plan_out, (cudaStream_t)stream);
+    return e == cudaSuccess ? TSENOR_OK : cuda_fail(e, "tsenor_plan launch");
+}
+
+extern "C" tsenor_status tsenor_round(const float* plan, const void* W, tsenor_dtype dtype, int64_t rows,
+                                      int64_t cols, int N, int M, int sweeps, uint32_t* mask_out,
+                                      tsenor_stream_t stream) {
+    tsenor_status s = check_common(W, dtype, rows, cols, N, M);
+    if (s != TSENOR_OK) return s;
+    if (sweeps < 0) return TSENOR_ERR_ARG;
+    if (rows == 0 || cols == 0) return TSENOR_OK;
+    if (!plan || !aligned(plan, 16) || !mask_out || !aligned(mask_out, 8)) return TSENOR_ERR_ARG;
+    cudaError_t e = run_round(dtype, M, plan, W, rows, cols, N, sweeps, mask_out, (cudaStream_t)stream);
+    return e == cudaSuccess ? TSENOR_OK : cuda_fail(e, "tsenor_round launch");
+}
+
+extern "C" tsenor_status tsenor_mask(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols, int N,
+                                     int M, float tau, int iters, int sweeps, uint32_t* mask_out,
+                                     tsenor_stream_t stream) {
+    tsenor_status s = check_common(W, dtype, rows, cols, N, M);
+    if (s != TSENOR_OK) return s;
+    if (!solver_params_ok(tau, iters) || sweeps < 0) return TSENOR_ERR_ARG;
+    if (rows == 0 || cols == 0) return TSENOR_OK;
+    if (!mask_out || !aligned(mask_out, 8)) return TSENOR_ERR_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    float* plan = nullptr;
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&plan), size_t(rows) * size_t(cols) * sizeof(float), st);
+    if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask workspace");
+    e = run_plan(dtype, M, W, rows, cols, N, tau, iters, plan, st);
+    if (e == cudaSuccess) e = run_round(dtype, M, plan, W, rows, cols, N, sweeps, mask_out, st);
+    cudaError_t e2 = cudaFreeAsync(plan, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask launch");
+    if (e2 != cudaSuccess) return cuda_fail(e2, "tsenor_mask workspace free");
+    return TSENOR_OK;
+}
+
+extern "C" tsenor_status tsenor_objective(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
+                                          const uint32_t* mask, int N, int M, double* out,
+                                          tsenor_stream_t stream) {
+    tsenor_status s = check_common(W, dtype, rows, cols, N, M);
+    if (s != TSENOR_OK) return s;
+    if (rows == 0 || cols == 0) return TSENOR_OK;
+    if (!mask || !out || !aligned(mask, 4) || !aligned(out, 8)) return TSENOR_ERR_ARG;
+    cudaError_t e = launch_objective(dtype == TSENOR_BF16, W, rows, cols, mask, N, M, out, (cudaStream_t)stream);
+    return e == cudaSuccess ? TSENOR_OK : cuda_fail(e, "tsenor_objective launch");
+}
+
+extern "C" tsenor_status tsenor_error_count(tsenor_stream_t stream, int64_t* count_out) {
+    if (!count_out) return TSENOR_ERR_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned long long v = 0;
+    const unsigned long long zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_block_failures, sizeof(v), 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaMemcpyToSymbolAsync(g_block_failures, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "tsenor_error_count");
+    *count_out = int64_t(v);
+    return TSENOR_OK;
+}
+
+extern "C" const char* tsenor_status_string(int status) {
+    switch (status) {
+        case TSENOR_OK: return "ok";
+        case TSENOR_ERR_ARG: return "invalid argument";
+        case TSENOR_ERR_SHAPE: return "rows/cols not a non-negative multiple of M";
+        case TSENOR_ERR_UNSUPPORTED_M: return "M must be 4, 8, 16, 32 or 64";
+        case TSENOR_ERR_CUDA: return "CUDA runtime error";
+        default: return "unknown status";
+    }
+}
+
+extern "C" const char* tsenor_last_error(void) { return tsenor::g_last_error; }

@@ -1,0 +1,80 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point that include/tsenor.h declares, and rejects bad arguments on the host
+before any CUDA call (no compute is run here)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import sparse_mask_search_b200 as tsl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(tsenor_[a-z_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    L = tsl.lib()
+    names = declared_functions()
+    assert set(tsl.EXPORTS) <= set(names) | {"tsenor_last_error"}
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings():
+    L = tsl.lib()
+    for code in (0, -1, -2, -3, -4):
+        assert L.tsenor_status_string(code)
+    assert L.tsenor_last_error() == b""
+
+
+def _mask(L, W=1 << 12, dtype=1, rows=64, cols=64, N=2, M=4, tau=10.0, iters=5, sweeps=1, out=1 << 12):
+    return L.tsenor_mask(W, dtype, rows, cols, N, M, tau, iters, sweeps, out, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(M=5), -3), (dict(M=128), -3), (dict(M=2), -3),
+    (dict(N=0), -1), (dict(N=5), -1),
+    (dict(rows=66), -2), (dict(cols=-4), -2),
+    (dict(tau=0.0), -1), (dict(tau=float("nan")), -1), (dict(tau=float("inf")), -1),
+    (dict(iters=0), -1), (dict(sweeps=-1), -1),
+    (dict(dtype=7), -1),
+    (dict(W=0), -1), (dict(W=(1 << 12) + 2), -1),
+    (dict(out=0), -1), (dict(out=(1 << 12) + 4), -1),
+])
+def test_host_side_argument_errors(kw, code):
+    assert _mask(tsl.lib(), **kw) == code
+
+
+def test_empty_calls_do_nothing():
+    L = tsl.lib()
+    assert _mask(L, rows=0, W=0, out=0) == 0
+    assert _mask(L, cols=0, W=0, out=0) == 0
+    assert L.tsenor_plan(0, 0, 0, 32, 2, 4, 1.0, 3, 0, None) == 0
+    assert L.tsenor_round(0, 0, 0, 32, 0, 2, 4, 1, 0, None) == 0
+    assert L.tsenor_objective(0, 0, 0, 0, 0, 2, 4, 0, None) == 0
+
+
+def test_other_entry_points_validate():
+    L = tsl.lib()
+    assert L.tsenor_plan(1 << 12, 1, 64, 64, 2, 4, 10.0, 5, 0, None) == -1        # no plan buffer
+    assert L.tsenor_plan(1 << 12, 1, 64, 64, 2, 6, 10.0, 5, 1 << 12, None) == -3
+    assert L.tsenor_round(1 << 12, 1 << 12, 1, 64, 64, 2, 4, -1, 1 << 12, None) == -1
+    assert L.tsenor_objective(1 << 12, 1, 64, 62, 1 << 12, 2, 4, 1 << 12, None) == -2
+    assert L.tsenor_error_count(None, None) == -1
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(tsl, "_lib", None)
+    monkeypatch.setattr(tsl, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        tsl.lib()
