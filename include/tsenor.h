@@ -61,7 +61,8 @@ typedef enum {
     TSENOR_ERR_ARG = -1,             /* null pointer, bad dtype, N/tau/iters/sweeps out of range, misaligned pointer */
     TSENOR_ERR_SHAPE = -2,           /* rows or cols negative or not a multiple of M */
     TSENOR_ERR_UNSUPPORTED_M = -3,   /* M not in {4, 8, 16, 32, 64} */
-    TSENOR_ERR_CUDA = -4             /* a CUDA runtime call failed; see tsenor_last_error() */
+    TSENOR_ERR_CUDA = -4,            /* a CUDA runtime call failed; see tsenor_last_error() */
+    TSENOR_ERR_TOO_LARGE = -5        /* tsenor_mask_noalloc: rows*cols above TSENOR_NOALLOC_MAX_PARAMS */
 } tsenor_status;
 
 /*
@@ -119,6 +120,43 @@ const char* tsenor_status_string(int status);
 
 /* Message of the last TSENOR_ERR_CUDA on the calling host thread ("" if none). */
 const char* tsenor_last_error(void);
+
+/*
+ * tsenor_mask_noalloc -- tsenor_mask for callers that must not allocate.
+ *
+ * The TSENOR review has no counterpart of this entry point; it exists for
+ * callers of this library that cannot let it allocate device memory:
+ *  - processes whose device memory is already reserved by another allocator
+ *    (for example a framework's caching allocator holding most of the GPU),
+ *    where a cudaMallocAsync inside the library can fail with out-of-memory
+ *    although the caller still has free space in its own pool;
+ *  - services that run under a fixed device-memory budget and must not grow
+ *    their footprint, or wait on an allocation, while they are serving.
+ *
+ * Same arguments, results and error behaviour as tsenor_mask; the only
+ * difference is where the plan between the two kernels lives.  Instead of a
+ * stream-ordered cudaMallocAsync workspace, it uses a file-scope device array
+ * of TSENOR_NOALLOC_MAX_PARAMS floats (64 MiB) inside the library.  That
+ * array exists on every GPU that loads the library and stays allocated until
+ * the process exits.  The call itself allocates nothing: no cudaMalloc,
+ * cudaMallocAsync, cudaFree or allocating library routine.
+ *
+ *  - rows * cols must not exceed TSENOR_NOALLOC_MAX_PARAMS; larger calls
+ *    return TSENOR_ERR_TOO_LARGE before anything is enqueued.
+ *  - The first call on a device looks up the array's device address on that
+ *    device (cudaGetSymbolAddress, with the device current) and keeps it for
+ *    later calls; make that first call before any stream capture.
+ *  - Every call on a device shares the one array, and the array keeps the
+ *    last call's contents.  Nothing in it needs to start at zero: each call
+ *    writes the whole plan region it later reads.  Calls whose work overlaps
+ *    on the GPU (different streams without ordering between them, or several
+ *    host threads) race on the array and corrupt each other's masks; order
+ *    them on one stream or with events.
+ */
+#define TSENOR_NOALLOC_MAX_PARAMS (16LL * 1024 * 1024)
+tsenor_status tsenor_mask_noalloc(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
+                                  int N, int M, float tau, int iters, int sweeps,
+                                  uint32_t* mask_out, tsenor_stream_t stream);
 
 #ifdef __cplusplus
 }

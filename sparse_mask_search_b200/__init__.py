@@ -14,9 +14,10 @@ LIB_PATH = os.path.join(HERE, "libtsenor_b200.so")
 
 TSENOR_F32, TSENOR_BF16 = 0, 1
 STATUS = {0: "TSENOR_OK", -1: "TSENOR_ERR_ARG", -2: "TSENOR_ERR_SHAPE", -3: "TSENOR_ERR_UNSUPPORTED_M",
-          -4: "TSENOR_ERR_CUDA"}
+          -4: "TSENOR_ERR_CUDA", -5: "TSENOR_ERR_TOO_LARGE"}
+NOALLOC_MAX_PARAMS = 16 * 1024 * 1024
 EXPORTS = ("tsenor_mask", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
-           "tsenor_status_string", "tsenor_last_error")
+           "tsenor_status_string", "tsenor_last_error", "tsenor_mask_noalloc")
 
 _lib = None
 
@@ -37,6 +38,7 @@ def lib() -> C.CDLL:
         L = C.CDLL(LIB_PATH)
         p, i64, i32, f32 = C.c_void_p, C.c_int64, C.c_int, C.c_float
         L.tsenor_mask.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p]
+        L.tsenor_mask_noalloc.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p]
         L.tsenor_plan.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, p, p]
         L.tsenor_round.argtypes = [p, p, i32, i64, i64, i32, i32, i32, p, p]
         L.tsenor_objective.argtypes = [p, i32, i64, i64, p, i32, i32, p, p]
@@ -96,6 +98,27 @@ def tsenor_mask(W, N: int, M: int, tau: float, iters: int, sweeps: int, out=None
     return out
 
 
+def tsenor_mask_noalloc(W, N: int, M: int, tau: float, iters: int, sweeps: int, out=None, stream=None):
+    """tsenor_mask without any device allocation by the library.
+
+    For callers whose device memory is reserved by another allocator or who
+    run under a fixed memory budget.  The plan between the two kernels lives
+    in a 64 MiB array inside the library (rows*cols <= NOALLOC_MAX_PARAMS).
+    All calls on a device share that array: calls that overlap on the GPU
+    race.  The first call on a device looks up the array's address; make it
+    before any stream capture.  Only ``out`` is allocated here (by torch)
+    when it is not given.
+    """
+    import torch
+    _check_2d_cuda(W, "W")
+    rows, cols = W.shape
+    if out is None:
+        out = torch.empty((rows, words_per_row(cols)), dtype=torch.int32, device=W.device)
+    _check(lib().tsenor_mask_noalloc(W.data_ptr(), _dtype_code(W), rows, cols, N, M, float(tau), iters,
+                                     sweeps, out.data_ptr(), _stream_handle(stream)))
+    return out
+
+
 def tsenor_plan(W, N: int, M: int, tau: float, iters: int, out=None, stream=None):
     """Fractional plan S (fp32, same shape as W) after `iters` Dykstra iterations."""
     import torch
@@ -142,5 +165,5 @@ def tsenor_error_count(stream=None) -> int:
     return int(n.value)
 
 
-__all__ = ["tsenor_mask", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
+__all__ = ["tsenor_mask", "tsenor_mask_noalloc", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
            "TsenorError", "lib", "words_per_row", "EXPORTS", "LIB_PATH"]

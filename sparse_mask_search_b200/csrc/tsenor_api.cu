@@ -2,6 +2,7 @@
 // dispatch on M and dtype, stream-ordered launches, the failure counter.
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <type_traits>
 
 #include "../../include/tsenor.h"
@@ -193,8 +194,60 @@ extern "C" const char* tsenor_status_string(int status) {
         case TSENOR_ERR_SHAPE: return "rows/cols not a non-negative multiple of M";
         case TSENOR_ERR_UNSUPPORTED_M: return "M must be 4, 8, 16, 32 or 64";
         case TSENOR_ERR_CUDA: return "CUDA runtime error";
+        case TSENOR_ERR_TOO_LARGE: return "rows*cols exceeds TSENOR_NOALLOC_MAX_PARAMS (16777216) of tsenor_mask_noalloc";
         default: return "unknown status";
     }
 }
 
 extern "C" const char* tsenor_last_error(void) { return tsenor::g_last_error; }
+
+// ---------------------------------------------------------------------------
+// tsenor_mask_noalloc: the plan between the two kernels lives in a file-scope
+// device array instead of a cudaMallocAsync workspace (see include/tsenor.h).
+// Host code must not hand `g_noalloc_plan` itself to a kernel: on the host
+// that name is only a stand-in for the symbol, not a device address.  The
+// device address is looked up once per device with cudaGetSymbolAddress.
+
+static __device__ __align__(256) float g_noalloc_plan[TSENOR_NOALLOC_MAX_PARAMS];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+float* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_plan on the current device (first call per device looks it up).
+cudaError_t noalloc_plan_ptr(float** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_plan);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = static_cast<float*>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+}  // namespace
+
+extern "C" tsenor_status tsenor_mask_noalloc(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols, int N,
+                                             int M, float tau, int iters, int sweeps, uint32_t* mask_out,
+                                             tsenor_stream_t stream) {
+    tsenor_status s = check_common(W, dtype, rows, cols, N, M);
+    if (s != TSENOR_OK) return s;
+    if (!solver_params_ok(tau, iters) || sweeps < 0) return TSENOR_ERR_ARG;
+    if (rows == 0 || cols == 0) return TSENOR_OK;
+    if (!mask_out || !aligned(mask_out, 8)) return TSENOR_ERR_ARG;
+    if (rows * cols > TSENOR_NOALLOC_MAX_PARAMS) return TSENOR_ERR_TOO_LARGE;
+    cudaStream_t st = (cudaStream_t)stream;
+    float* plan = nullptr;
+    cudaError_t e = noalloc_plan_ptr(&plan);
+    if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask_noalloc device array address");
+    e = run_plan(dtype, M, W, rows, cols, N, tau, iters, plan, st);
+    if (e == cudaSuccess) e = run_round(dtype, M, plan, W, rows, cols, N, sweeps, mask_out, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask_noalloc launch");
+    return TSENOR_OK;
+}
