@@ -25,6 +25,28 @@ __device__ __forceinline__ float rcp(float x) {
     return y;
 }
 
+// Packed fp32 pairs (PTX f32x2, sm_100): two adds / multiplies / fmas per
+// instruction, round to nearest even per element.
+union F2U {
+    float2 f;
+    unsigned long long u;
+};
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    F2U x{a}, y{b}, d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d.u) : "l"(x.u), "l"(y.u));
+    return d.f;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    F2U x{a}, y{b}, d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.u) : "l"(x.u), "l"(y.u));
+    return d.f;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    F2U x{a}, y{b}, z{c}, d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.u) : "l"(x.u), "l"(y.u), "l"(z.u));
+    return d.f;
+}
+
 // Element types of W.  Loads return |W| as fp32 (exact for both types).
 struct F32 {
     using storage = float;

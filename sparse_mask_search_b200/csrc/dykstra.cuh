@@ -25,6 +25,9 @@ namespace tsenor {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Plan entry of one state value: S = 2^min(y, 0), exactly 1 when clipped.
+__device__ __forceinline__ float plan_value(float y) { return y >= 0.f ? 1.f : ex2(y); }
+
 // ---------------------------------------------------------------------------
 // M = 4, 8: one thread holds a whole block in registers.  Rows are streamed:
 // the exponentials of one row live only until its column contributions are
@@ -104,7 +107,7 @@ dykstra_thread_kernel(const typename T::storage* __restrict__ W, int64_t cols, i
         float s[M];
 #pragma unroll
         for (int j = 0; j < M; ++j)
-            s[j] = !finite ? __int_as_float(0x7fc00000) : (y[i][j] >= 0.f ? 1.f : ex2(y[i][j]));
+            s[j] = !finite ? __int_as_float(0x7fc00000) : plan_value(y[i][j]);
         float* dst = plan + (r0 + i) * cols + c0;
 #pragma unroll
         for (int v = 0; v < M / 4; ++v)
@@ -146,33 +149,47 @@ struct TileCfg {
     static_assert(CG * RSC == 32 || WC == 1, "cross-warp columns need full warps");
 };
 
-template <int M, typename T>
-__global__ void __launch_bounds__(128)
-dykstra_tile_kernel(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks,
-                    int N, float tau, int iters, float* __restrict__ plan) {
+// Identity of a thread inside its block's tile, and the permuted local row /
+// column that its register k / c holds.
+template <int M>
+struct TileThread {
+    using C = TileCfg<M>;
+    int tid, lane, warp, blk, t, cg, rg, gr, gc;
+    __device__ __forceinline__ TileThread() {
+        tid = threadIdx.x;
+        lane = tid & 31;
+        warp = tid >> 5;
+        blk = tid / C::TPB;            // block slot within the CTA
+        t = tid % C::TPB;              // thread within the block
+        cg = t % C::CG;
+        rg = t / C::CG;
+        gr = cg % C::RSR;              // index in the row reduce-scatter group
+        gc = rg % C::RSC;              // index in the column reduce-scatter group
+    }
+    __device__ __forceinline__ int lrow(int k) const { return ((k / C::RO) ^ gr) * C::RO + (k % C::RO); }
+    __device__ __forceinline__ int lcol(int c) const { return ((c / C::CO) ^ gc) * C::CO + (c % C::CO); }
+    __device__ __forceinline__ int row(int k) const { return C::P * rg + lrow(k); }   // row within the block
+    __device__ __forceinline__ int col(int c) const { return C::Q * cg + lcol(c); }   // column within the block
+};
+
+// Dykstra for one block spread over its TPB threads.  On return `y` holds the
+// final state of this thread's sub-tile and `tile` the block's |W| (M x M in
+// shared memory, row stride TS).  Contains CTA-wide barriers: every thread of the CTA
+// must call it.  Returns whether the block's W is finite.
+template <int M, typename T, int TS = M>
+__device__ __forceinline__ bool dykstra_tile_solve(const typename T::storage* __restrict__ W, int64_t cols,
+                                                   int64_t r0, int64_t c0, bool active, int N, float tau,
+                                                   int iters, float* tile, float* colbuf,
+                                                   const TileThread<M>& th, float (&y)[4][8]) {
     using C = TileCfg<M>;
     constexpr int P = C::P, Q = C::Q;
-    extern __shared__ float smem[];
-    // tile staging: one M x M float tile per block of the CTA
-    float* tiles = smem;
-    float* colbuf = smem + C::BPC * M * M;   // [2][warps][32][CO] for cross-warp columns
-
-    const int tid = threadIdx.x;
-    const int lane = tid & 31, warp = tid >> 5;
-    const int blk = tid / C::TPB;                  // block slot within the CTA
-    const int t = tid % C::TPB;                    // thread within the block
-    const int cg = t % C::CG, rg = t / C::CG;
-    const int64_t b = int64_t(blockIdx.x) * C::BPC + blk;
-    const bool active = b < n_blocks;
-    const int64_t nbc = cols / M;
-    const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
-    float* tile = tiles + blk * M * M;
+    const int lane = th.lane, warp = th.warp;
 
     // ---- stage |W| of the block in shared memory (16-byte coalesced loads)
     {
         constexpr int V = T::kVec;
         constexpr int CPR = M / V;                 // 16-byte chunks per tile row
-        for (int q = t; q < M * CPR; q += C::TPB) {
+        for (int q = th.t; q < M * CPR; q += C::TPB) {
             const int i = q / CPR, v = q % CPR;
             float tmp[V];
             if (active) T::load16(W + (r0 + i) * cols + c0 + v * V, tmp);
@@ -181,25 +198,18 @@ dykstra_tile_kernel(const typename T::storage* __restrict__ W, int64_t cols, int
                 for (int u = 0; u < V; ++u) tmp[u] = 0.f;
             }
 #pragma unroll
-            for (int u = 0; u < V; ++u) tile[i * M + v * V + u] = tmp[u];
+            for (int u = 0; u < V; ++u) tile[i * TS + v * V + u] = tmp[u];
         }
     }
     __syncthreads();
 
-    // permuted local row / column of register k / c
-    const int gr = cg % C::RSR;                     // index in the row reduce-scatter group
-    const int gc = rg % C::RSC;                     // index in the column reduce-scatter group
-    auto lrow = [&](int k) { return ((k / C::RO) ^ gr) * C::RO + (k % C::RO); };
-    auto lcol = [&](int c) { return ((c / C::CO) ^ gc) * C::CO + (c % C::CO); };
-
-    float y[P][Q];
     float m = 0.f;
     bool finite = true;
 #pragma unroll
     for (int k = 0; k < P; ++k)
 #pragma unroll
         for (int c = 0; c < Q; ++c) {
-            const float a = tile[(P * rg + lrow(k)) * M + Q * cg + lcol(c)];
+            const float a = tile[th.row(k) * TS + th.col(c)];
             y[k][c] = a;
             finite = finite && (a <= 3.402823466e38f);
             m = fmaxf(m, a);
@@ -236,20 +246,26 @@ dykstra_tile_kernel(const typename T::storage* __restrict__ W, int64_t cols, int
 
     // Blocks of one warp (M = 16) may differ in finiteness; all lanes run the
     // loop so that the shuffles stay converged, and a non-finite block's
-    // result is replaced by NaN at the end.
+    // result is discarded by the caller.
+    // Column pairs (c, c+1) of a row are handled as packed fp32x2 values.
+    constexpr int Q2 = Q / 2;
+    float2 y2[P][Q2];
+#pragma unroll
+    for (int k = 0; k < P; ++k)
+#pragma unroll
+        for (int c = 0; c < Q2; ++c) y2[k][c] = make_float2(y[k][2 * c], y[k][2 * c + 1]);
     const bool run = (C::TPB <= 32) ? (__any_sync(kFullMask, finite) != 0) : finite;
     if (run) {
         for (int it = 0; it < iters; ++it) {
-            float e[P][Q];
+            float2 e2[P][Q2];
             float rs[P];
 #pragma unroll
             for (int k = 0; k < P; ++k) {
-                rs[k] = 0.f;
 #pragma unroll
-                for (int c = 0; c < Q; ++c) {
-                    e[k][c] = ex2(fminf(y[k][c], 0.f));
-                    rs[k] += e[k][c];
-                }
+                for (int c = 0; c < Q2; ++c)
+                    e2[k][c] = make_float2(ex2(fminf(y2[k][c].x, 0.f)), ex2(fminf(y2[k][c].y, 0.f)));
+                const float2 acc = add2(add2(e2[k][0], e2[k][1]), add2(e2[k][2], e2[k][3]));
+                rs[k] = acc.x + acc.y;
             }
             // row reduce-scatter over RSR lanes, then all-reduce over ARR
 #pragma unroll
@@ -284,11 +300,12 @@ dykstra_tile_kernel(const typename T::storage* __restrict__ W, int64_t cols, int
             // column partial sums of e * w
             float cs[Q];
 #pragma unroll
-            for (int c = 0; c < Q; ++c) {
-                float acc = e[0][c] * wv[0];
+            for (int c = 0; c < Q2; ++c) {
+                float2 acc = mul2(e2[0][c], make_float2(wv[0], wv[0]));
 #pragma unroll
-                for (int k = 1; k < P; ++k) acc = fmaf(e[k][c], wv[k], acc);
-                cs[c] = acc;
+                for (int k = 1; k < P; ++k) acc = fma2(e2[k][c], make_float2(wv[k], wv[k]), acc);
+                cs[2 * c] = acc.x;
+                cs[2 * c + 1] = acc.y;
             }
 #pragma unroll
             for (int s = C::RSC / 2; s >= 1; s >>= 1)
@@ -320,26 +337,52 @@ dykstra_tile_kernel(const typename T::storage* __restrict__ W, int64_t cols, int
 #pragma unroll
                     for (int lo = 0; lo < C::CO; ++lo)
                         cv[(hi + s) * C::CO + lo] = __shfl_xor_sync(kFullMask, cv[hi * C::CO + lo], s * C::CG);
+            // y += r_i + c_j
 #pragma unroll
             for (int k = 0; k < P; ++k)
 #pragma unroll
-                for (int c = 0; c < Q; ++c) y[k][c] += rv[k] + cv[c];
+                for (int c = 0; c < Q2; ++c)
+                    y2[k][c] = add2(y2[k][c], add2(make_float2(rv[k], rv[k]), make_float2(cv[2 * c], cv[2 * c + 1])));
         }
     }
-
-    // ---- plan S = 2^min(y,0) (1 exactly when clipped), via the smem tile
-    __syncthreads();
 #pragma unroll
     for (int k = 0; k < P; ++k)
 #pragma unroll
-        for (int c = 0; c < Q; ++c) {
-            const float s = !finite ? __int_as_float(0x7fc00000) : (y[k][c] >= 0.f ? 1.f : ex2(y[k][c]));
-            tile[(P * rg + lrow(k)) * M + Q * cg + lcol(c)] = s;
+        for (int c = 0; c < Q2; ++c) {
+            y[k][2 * c] = y2[k][c].x;
+            y[k][2 * c + 1] = y2[k][c].y;
         }
+    return finite;
+}
+
+template <int M, typename T>
+__global__ void __launch_bounds__(128)
+dykstra_tile_kernel(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks,
+                    int N, float tau, int iters, float* __restrict__ plan) {
+    using C = TileCfg<M>;
+    extern __shared__ float smem[];
+    const TileThread<M> th;
+    float* tile = smem + th.blk * M * M;
+    float* colbuf = smem + C::BPC * M * M;         // [2][warps][32][CO] for cross-warp columns
+    const int64_t b = int64_t(blockIdx.x) * C::BPC + th.blk;
+    const bool active = b < n_blocks;
+    const int64_t nbc = cols / M;
+    const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
+
+    float y[C::P][C::Q];
+    const bool finite = dykstra_tile_solve<M, T>(W, cols, r0, c0, active, N, tau, iters, tile, colbuf, th, y);
+
+    // ---- plan via the smem tile, then 16-byte coalesced stores
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < C::P; ++k)
+#pragma unroll
+        for (int c = 0; c < C::Q; ++c)
+            tile[th.row(k) * M + th.col(c)] = finite ? plan_value(y[k][c]) : __int_as_float(0x7fc00000);
     __syncthreads();
     if (active) {
         constexpr int CPR = M / 4;
-        for (int q = t; q < M * CPR; q += C::TPB) {
+        for (int q = th.t; q < M * CPR; q += C::TPB) {
             const int i = q / CPR, v = q % CPR;
             const float4 val = *reinterpret_cast<const float4*>(tile + i * M + 4 * v);
             *reinterpret_cast<float4*>(plan + (r0 + i) * cols + c0 + 4 * v) = val;

@@ -1,0 +1,638 @@
+// Rounding of one block's fractional plan into a transposable N:M mask by one
+// warp ("What carries the argument" and the Fig. 2 caption of the TSENOR
+// review; referee comment 3 on the rounding stage).
+//
+//   1. sort: each lane holds R = E/32 keys in registers (E = M*M, padded to
+//      32 for M = 4); a bitonic network orders them so that position
+//      p = lane*R + r holds the p-th entry of the rounding order (plan desc,
+//      |W| desc, flat index asc).  Distances below R are compare-exchanges
+//      inside a lane, larger ones are shuffles between lanes;
+//   2. greedy: entries in sorted order are taken while their row and column
+//      budgets N remain.  The warp decides 32 consecutive entries at a time;
+//      a lane is settled as soon as an upper bound (all undecided earlier
+//      lanes of its row/column taken) keeps it within budget, or a lower bound
+//      (only accepted earlier lanes) exhausts it.  The first undecided lane is
+//      always settled, so the result is exactly the sequential greedy;
+//   3. repair: while a row is short, the lowest short row i and lowest short
+//      column j get the 2-in/1-out move (i,j'),(i',j) in, (i',j') out with the
+//      best score (a_ij' + a_i'j) - a_i'j' of any sign (ties: lowest i'*M+j');
+//   4. local search: anchors i = 0..M-1 per sweep; the partner i' with the
+//      best net gain max_{j in O_i\O_i'}(a_i'j - a_ij) + max_{j' in O_i'\O_i}
+//      (a_ij' - a_i'j') is swapped when that gain is positive.  The gain of a
+//      row pair depends on those two rows only and is symmetric, so it is
+//      cached in an M x M table and only the two rows touched by a swap are
+//      recomputed; once M anchors in a row found nothing the state is a fixed
+//      point and the remaining sweeps are skipped (they would change nothing);
+//   5. the caller writes the row bitmasks.
+// Every comparison that decides an integer uses fp32 values evaluated in the
+// order written above.
+#pragma once
+
+#include <climits>
+
+#include "common.cuh"
+
+namespace tsenor {
+
+__device__ unsigned long long g_block_failures;   // blocks that could not be rounded
+
+// Sort keys.  KeyB (bf16 input): the low 16 bits of |W| are zero, so one
+// 64-bit word holds plan bits, |W| bits and the complemented index:
+// a larger word is earlier in the rounding order.  KeyF (fp32 input): plan and
+// |W| bits in one word, the index in a second one.
+struct KeyB {
+    unsigned long long k;
+    __device__ __forceinline__ static KeyB make(float s, float a, int idx) {
+        return KeyB{(static_cast<unsigned long long>(__float_as_uint(s)) << 32) |
+                    (__float_as_uint(a) & 0xffff0000u) | (0xffffu - static_cast<unsigned>(idx))};
+    }
+    __device__ __forceinline__ static KeyB sentinel() { return KeyB{0ull}; }
+    __device__ __forceinline__ int index() const { return int(0xffffu - unsigned(k & 0xffffu)); }
+    __device__ __forceinline__ bool before(const KeyB& o) const { return k > o.k; }
+    __device__ __forceinline__ KeyB shfl_xor(int m) const {
+        return KeyB{__shfl_xor_sync(kFullMask, k, m)};
+    }
+};
+
+struct KeyF {
+    unsigned long long k;
+    unsigned idx;
+    __device__ __forceinline__ static KeyF make(float s, float a, int idx) {
+        return KeyF{(static_cast<unsigned long long>(__float_as_uint(s)) << 32) | __float_as_uint(a),
+                    static_cast<unsigned>(idx)};
+    }
+    __device__ __forceinline__ static KeyF sentinel() { return KeyF{0ull, 0xffffffffu}; }
+    __device__ __forceinline__ int index() const { return int(idx); }
+    __device__ __forceinline__ bool before(const KeyF& o) const { return k > o.k || (k == o.k && idx < o.idx); }
+    __device__ __forceinline__ KeyF shfl_xor(int m) const {
+        return KeyF{__shfl_xor_sync(kFullMask, k, m), __shfl_xor_sync(kFullMask, idx, m)};
+    }
+};
+
+template <typename T> struct KeyOf;
+template <> struct KeyOf<BF16> { using type = KeyB; };
+template <> struct KeyOf<F32> { using type = KeyF; };
+
+template <int M>
+struct WarpRound {
+    static constexpr int E = M * M;
+    static constexpr int EP = E < 32 ? 32 : E;     // padded entry count
+    static constexpr int R = EP / 32;              // keys per lane (M <= 32)
+    static constexpr int AS = M + 1;               // row stride of |W| and of the gain table in smem
+    using Bits = typename std::conditional<(M > 32), unsigned long long, unsigned>::type;   // one row
+};
+
+template <typename Bits>
+__device__ __forceinline__ int lowest_bit(Bits x) {
+    if constexpr (sizeof(Bits) == 8) return __ffsll(static_cast<long long>(x)) - 1;
+    else return __ffs(static_cast<int>(x)) - 1;
+}
+
+// Per-block shared memory of the rounding steps after the sort.
+template <int M>
+struct RoundShared {
+    using Bits = typename WarpRound<M>::Bits;
+    static constexpr int GS = M + 1;
+    float G[M * GS];                    // cached pair gains (local search), row stride M+1
+    uint16_t order[WarpRound<M>::EP];   // sorted flat indices
+    Bits rowbits[M];
+    float bestv[M];                     // best gain of each row over its partners ...
+    int bestp[M];                       // ... and that partner (lowest index on ties)
+    int rc[M];
+    int cc[M];
+};
+
+// Bitonic compare-exchange of registers r and r|J of this lane: the pair ends
+// earliest-first when `up`.  The order is strict (no two keys of a block are
+// equal), so one comparison decides either direction.
+template <int R, int J, typename Key>
+__device__ __forceinline__ void bitonic_regs(Key (&key)[R], bool up) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        if (r & J) continue;
+        const Key x = key[r], y = key[r | J];
+        const bool sw = y.before(x) == up;
+        key[r] = sw ? y : x;
+        key[r | J] = sw ? x : y;
+    }
+}
+
+// In-register stages j = J, J/2, ..., 1 with a direction that is constant
+// over this lane's registers.
+template <int R, int J, typename Key>
+__device__ __forceinline__ void bitonic_regs_down(Key (&key)[R], bool up) {
+    if constexpr (J >= 1) {
+        bitonic_regs<R, J>(key, up);
+        bitonic_regs_down<R, J / 2>(key, up);
+    }
+}
+
+// Phase 1 of the sort: each lane's R registers (positions lane*R + r) become a
+// sorted run, earliest-first on even lanes and latest-first on odd lanes.
+template <int R, int K, typename Key>
+__device__ __forceinline__ void bitonic_local(Key (&key)[R], int lane) {
+    if constexpr (K <= R) {
+#pragma unroll
+        for (int j = K / 2; j >= 1; j >>= 1) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                if (r & j) continue;
+                const bool up = K < R ? ((r & K) == 0) : ((lane & 1) == 0);
+                const Key x = key[r], y = key[r | j];
+                const bool sw = y.before(x) == up;
+                key[r] = sw ? y : x;
+                key[r | j] = sw ? x : y;
+            }
+        }
+        bitonic_local<R, K * 2>(key, lane);
+    }
+}
+
+// Cross-lane stage: pair lane with lane ^ m, same register.
+template <int R, typename Key>
+__device__ __forceinline__ void bitonic_shfl(Key (&key)[R], int m, bool take_earlier) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const Key x = key[r];
+        const Key y = x.shfl_xor(m);
+        key[r] = (y.before(x) == take_earlier) ? y : x;
+    }
+}
+
+// Bitonic sort of 32*R keys held R per lane (position p = lane*R + r),
+// earliest first.  Distances below R are compare-exchanges inside a lane,
+// larger ones pair lane with lane ^ (j/R) through shuffles.
+template <int R, typename Key>
+__device__ __forceinline__ void warp_bitonic_sort(Key (&key)[R], int lane) {
+    constexpr int EP = 32 * R;
+    bitonic_local<R, 2>(key, lane);
+#pragma unroll 1
+    for (int k = 2 * R; k <= EP; k <<= 1) {
+        const bool up = ((lane * R) & k) == 0;       // same for all of this lane's positions
+#pragma unroll 1
+        for (int j = k >> 1; j >= R; j >>= 1) {
+            const int m = j / R;
+            bitonic_shfl<R>(key, m, ((lane & m) == 0) == up);
+        }
+        bitonic_regs_down<R, R / 2>(key, up);
+    }
+}
+
+// Bitonic sort of 4096 keys over a CTA of 4 warps (M = 64): 32 keys per
+// thread at position t*32 + r (t = warp*32 + lane).  Distances of a warp's
+// 1024 positions or more go through shared memory (xbuf: 4*32*32 keys).
+template <typename Key>
+__device__ void cta_bitonic_sort64(Key (&key)[32], Key* xbuf, int warp, int lane) {
+    constexpr int R = 32, EP = 4096;
+    const int t = warp * 32 + lane;
+    bitonic_local<R, 2>(key, lane);
+#pragma unroll 1
+    for (int k = 2 * R; k <= EP; k <<= 1) {
+        const bool up = ((t * R) & k) == 0;
+#pragma unroll 1
+        for (int j = k >> 1; j >= R; j >>= 1) {
+            if (j >= 32 * R) {
+                const int mw = j / (32 * R);
+#pragma unroll
+                for (int r = 0; r < R; ++r) xbuf[(warp * R + r) * 32 + lane] = key[r];
+                __syncthreads();
+                const bool take_earlier = ((warp & mw) == 0) == up;
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const Key x = key[r];
+                    const Key y = xbuf[((warp ^ mw) * R + r) * 32 + lane];
+                    key[r] = (y.before(x) == take_earlier) ? y : x;
+                }
+                __syncthreads();
+            } else {
+                const int m = j / R;
+                bitonic_shfl<R>(key, m, ((lane & m) == 0) == up);
+            }
+        }
+        bitonic_regs_down<R, R / 2>(key, up);
+    }
+}
+
+__device__ __forceinline__ void warp_argmax(float& v, int& i) {
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) {
+        const float ov = __shfl_xor_sync(kFullMask, v, s);
+        const int oi = __shfl_xor_sync(kFullMask, i, s);
+        if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
+    }
+}
+
+// Sorted keys of one warp into sh.order.
+template <int M, typename Key>
+__device__ __forceinline__ void keys_to_order(const Key (&key)[WarpRound<M>::R], RoundShared<M>& sh, int lane) {
+    constexpr int R = WarpRound<M>::R, E = M * M;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int idx = key[r].index();
+        sh.order[lane * R + r] = static_cast<uint16_t>(idx < E ? idx : 0xffff);
+    }
+}
+
+// Steps 2-3 (greedy, repair) for one block by one warp, from sh.order.
+// Returns false when the block could not be made feasible.
+template <int M, int EP>
+__device__ bool greedy_and_repair(const float* a, RoundShared<M>& sh, int N, int lane) {
+    using Bits = typename WarpRound<M>::Bits;
+    constexpr int E = M * M, AS = M + 1;
+    for (int r = lane; r < M; r += 32) { sh.rc[r] = 0; sh.cc[r] = 0; sh.rowbits[r] = 0; }
+    __syncwarp();
+    const int target = N * M;
+    int taken = 0;
+    for (int base = 0; base < EP && taken < target; base += 32) {
+        const int e = sh.order[base + lane];
+        const bool valid = e < E;
+        const int i = valid ? e / M : 0, j = valid ? e % M : 0;
+        const unsigned mr = __match_any_sync(kFullMask, valid ? i : 4096 + lane);
+        const unsigned mc = __match_any_sync(kFullMask, valid ? j : 8192 + lane);
+        const unsigned lt = (1u << lane) - 1u;
+        const int r0c = valid ? sh.rc[i] : N, c0c = valid ? sh.cc[j] : N;
+        unsigned acc = 0u;
+        unsigned und = __ballot_sync(kFullMask, valid && r0c < N && c0c < N);
+        while (und) {
+            const bool mine = (und >> lane) & 1u;
+            const unsigned maybe = acc | und;
+            const int ru = r0c + __popc(mr & lt & maybe), cu = c0c + __popc(mc & lt & maybe);
+            const int rl = r0c + __popc(mr & lt & acc), cl = c0c + __popc(mc & lt & acc);
+            const unsigned A = __ballot_sync(kFullMask, mine && ru < N && cu < N);
+            const unsigned Rj = __ballot_sync(kFullMask, mine && (rl >= N || cl >= N));
+            acc |= A;
+            und &= ~(A | Rj);
+        }
+        const bool mine_acc = (acc >> lane) & 1u;
+        // accepted entries set their bit (32-bit shared atomics); the lowest
+        // accepted lane of each row (column) group adds the group's count
+        if (mine_acc) atomicOr(reinterpret_cast<unsigned*>(&sh.rowbits[i]) + (j >> 5), 1u << (j & 31));
+        const unsigned ga = mr & acc, gc = mc & acc;
+        if (ga && __ffs(ga) - 1 == lane) sh.rc[i] += __popc(ga);
+        if (gc && __ffs(gc) - 1 == lane) sh.cc[j] += __popc(gc);
+        taken += __popc(acc);
+        __syncwarp();
+    }
+
+    for (int guard = 0; guard <= target; ++guard) {
+        unsigned long long shortR, shortC;
+        if constexpr (M <= 32) {
+            shortR = __ballot_sync(kFullMask, lane < M && sh.rc[lane] < N);
+            shortC = __ballot_sync(kFullMask, lane < M && sh.cc[lane] < N);
+        } else {
+            shortR = __ballot_sync(kFullMask, sh.rc[lane] < N) |
+                     (static_cast<unsigned long long>(__ballot_sync(kFullMask, sh.rc[lane + 32] < N)) << 32);
+            shortC = __ballot_sync(kFullMask, sh.cc[lane] < N) |
+                     (static_cast<unsigned long long>(__ballot_sync(kFullMask, sh.cc[lane + 32] < N)) << 32);
+        }
+        if (!shortR) return true;
+        if (!shortC || guard == target) return false;
+        const int i = __ffsll((long long)shortR) - 1, j = __ffsll((long long)shortC) - 1;
+        const Bits Oi = sh.rowbits[i];
+        float best = -INFINITY;
+        int bflat = INT_MAX;
+        for (int ip = lane; ip < M; ip += 32) {
+            const Bits Op = sh.rowbits[ip];
+            if ((Op >> j) & 1) continue;
+            Bits cand = Op & ~Oi;
+            while (cand) {
+                const int jp = lowest_bit(cand);
+                cand &= cand - 1;
+                const float sigma = __fsub_rn(__fadd_rn(a[i * AS + jp], a[ip * AS + j]), a[ip * AS + jp]);
+                const int flat = ip * M + jp;
+                if (sigma > best || (sigma == best && flat < bflat)) { best = sigma; bflat = flat; }
+            }
+        }
+        warp_argmax(best, bflat);
+        if (bflat == INT_MAX) return false;
+        if (lane == 0) {
+            const int ip = bflat / M, jp = bflat % M;
+            sh.rowbits[i] |= Bits(1) << jp;
+            sh.rowbits[ip] = (sh.rowbits[ip] | (Bits(1) << j)) & ~(Bits(1) << jp);
+            sh.rc[i] += 1;
+            sh.cc[j] += 1;
+        }
+        __syncwarp();
+    }
+    return false;
+}
+
+// Thread layout of the local search: NT threads (one warp for M <= 32, a CTA
+// of 4 warps for M = 64); thread tid serves partner row y = tid / CH and
+// columns [h*CPT, (h+1)*CPT) of it, h = tid % CH.  Each thread keeps those
+// |W| values of its row in registers.
+template <int M>
+struct LsCfg {
+    static constexpr int NT = M <= 32 ? 32 : 128;
+    static constexpr int CH = M <= 32 ? 1 : 2;      // threads per row
+    static constexpr int CPT = M / CH;              // columns per thread
+};
+
+template <int NT>
+__device__ __forceinline__ void ls_barrier() {
+    if constexpr (NT == 32) __syncwarp(); else __syncthreads();
+}
+
+// Pair gain pieces of row y against row x over this thread's columns:
+// txy = max over j in O_x \ O_y of (a_yj - a_xj), tyx = max over j in O_y \ O_x
+// of (a_xj - a_yj); the net gain of the exchange is txy + tyx (item 4 above).
+template <int M, int CPT, typename Bits>
+__device__ __forceinline__ void pair_pieces(const float (&ay)[CPT], const float* ax, Bits Ox, Bits Oy, int j0,
+                                            float& txy, float& tyx) {
+    const Bits m1 = Ox & ~Oy, m2 = Oy & ~Ox;
+#pragma unroll
+    for (int jj = 0; jj < CPT; ++jj) {
+        const int j = j0 + jj;
+        const float d = __fsub_rn(ay[jj], ax[j]);
+        if ((m1 >> j) & 1) txy = fmaxf(txy, d);
+        if ((m2 >> j) & 1) tyx = fmaxf(tyx, -d);
+    }
+}
+
+template <int CH>
+__device__ __forceinline__ float row_max(float t) {
+#pragma unroll
+    for (int s = 1; s < CH; s <<= 1) t = fmaxf(t, __shfl_xor_sync(kFullMask, t, s));
+    return t;
+}
+
+// Best partner of row x over the cached gains (lowest partner index on ties).
+template <int M>
+__device__ __forceinline__ void rescan_row(RoundShared<M>& sh, int x) {
+    constexpr int GS = M + 1;
+    float g[M];
+#pragma unroll
+    for (int y = 0; y < M; ++y) g[y] = sh.G[x * GS + y];
+    float bv = -INFINITY;
+    int bp = -1;
+#pragma unroll
+    for (int y = 0; y < M; ++y) {
+        if (y == x) continue;
+        if (bp < 0 || g[y] > bv) { bv = g[y]; bp = y; }
+    }
+    sh.bestv[x] = bv;
+    sh.bestp[x] = bp;
+}
+
+// Step 4 for one block by LsCfg<M>::NT threads: the gain table, the row
+// bests, then the sweeps.  `a`: |W| with row stride M+1.
+template <int M>
+__device__ void local_search(const float* a, RoundShared<M>& sh, int sweeps, int tid) {
+    using L = LsCfg<M>;
+    using Bits = typename WarpRound<M>::Bits;
+    constexpr int AS = M + 1, GS = M + 1, NT = L::NT, CH = L::CH, CPT = L::CPT;
+    const int lane = tid & 31;
+    const int y = tid / CH, h = tid % CH, j0 = h * CPT;
+    const bool row_thread = y < M;
+    float ay[CPT];
+#pragma unroll
+    for (int jj = 0; jj < CPT; ++jj) ay[jj] = row_thread ? a[y * AS + j0 + jj] : 0.f;
+
+    // gain table: row y with rows y+1 .. y+M/2 (mod M), every unordered pair once
+    {
+        const Bits Oy = row_thread ? sh.rowbits[y] : Bits(0);
+#pragma unroll 1
+        for (int d = 1; d <= M / 2; ++d) {
+            const int x = (y + d) & (M - 1);
+            float txy = -INFINITY, tyx = -INFINITY;
+            if (row_thread) pair_pieces<M, CPT, Bits>(ay, a + x * AS, sh.rowbits[x], Oy, j0, txy, tyx);
+            txy = row_max<CH>(txy);
+            tyx = row_max<CH>(tyx);
+            if (row_thread && h == 0 && !(d == M / 2 && y >= M / 2)) {
+                const float g = __fadd_rn(txy, tyx);
+                sh.G[x * GS + y] = g;
+                sh.G[y * GS + x] = g;
+            }
+        }
+    }
+    ls_barrier<NT>();
+    if (row_thread && h == 0) rescan_row<M>(sh, y);
+    ls_barrier<NT>();
+
+    int quiet = 0;                                   // anchors in a row without a swap
+    for (int sw = 0; sw < sweeps && quiet < M; ++sw) {
+        for (int i = 0; i < M && quiet < M; ++i) {
+            const float best = sh.bestv[i];
+            const int bp = sh.bestp[i];
+            if (!(best > 0.f)) { ++quiet; continue; }
+            const Bits Oi = sh.rowbits[i], Ob = sh.rowbits[bp];
+            // entries to exchange (every warp finds the same pair): lowest index on ties
+            float v1 = -INFINITY, v2 = -INFINITY;
+            int j1 = INT_MAX, j2 = INT_MAX;
+            for (int jj = lane; jj < M; jj += 32) {
+                const bool in_i = (Oi >> jj) & 1, in_p = (Ob >> jj) & 1;
+                if (in_i && !in_p) {
+                    const float d = __fsub_rn(a[bp * AS + jj], a[i * AS + jj]);
+                    if (j1 == INT_MAX || d > v1) { v1 = d; j1 = jj; }
+                }
+                if (!in_i && in_p) {
+                    const float d = __fsub_rn(a[i * AS + jj], a[bp * AS + jj]);
+                    if (j2 == INT_MAX || d > v2) { v2 = d; j2 = jj; }
+                }
+            }
+            warp_argmax(v1, j1);
+            warp_argmax(v2, j2);
+            if (j1 >= M || j2 >= M) { ++quiet; continue; }   // unreachable: a positive gain needs both sets
+            quiet = 0;
+            const Bits Oi2 = (Oi & ~(Bits(1) << j1)) | (Bits(1) << j2);
+            const Bits Ob2 = (Ob & ~(Bits(1) << j2)) | (Bits(1) << j1);
+            const Bits Oy = !row_thread ? Bits(0) : (y == i) ? Oi2 : (y == bp) ? Ob2 : sh.rowbits[y];
+            ls_barrier<NT>();                        // everyone has read the old rows
+            if (tid == 0) {
+                sh.rowbits[i] = Oi2;
+                sh.rowbits[bp] = Ob2;
+            }
+            // new gains g(i, y) and g(bp, y) of partner row y
+            float t1i = -INFINITY, t2i = -INFINITY, t1b = -INFINITY, t2b = -INFINITY;
+            if (row_thread) {
+                pair_pieces<M, CPT, Bits>(ay, a + i * AS, Oi2, Oy, j0, t1i, t2i);
+                pair_pieces<M, CPT, Bits>(ay, a + bp * AS, Ob2, Oy, j0, t1b, t2b);
+            }
+            t1i = row_max<CH>(t1i); t2i = row_max<CH>(t2i);
+            t1b = row_max<CH>(t1b); t2b = row_max<CH>(t2b);
+            const float gi = __fadd_rn(t1i, t2i), gb = __fadd_rn(t1b, t2b);
+            if (row_thread && h == 0) {
+                if (y != i) { sh.G[i * GS + y] = gi; sh.G[y * GS + i] = gi; }
+                if (y != i && y != bp) { sh.G[bp * GS + y] = gb; sh.G[y * GS + bp] = gb; }
+            }
+            ls_barrier<NT>();                        // gain table and rows complete
+            if (row_thread && h == 0) {
+                const int op = sh.bestp[y];
+                if (y == i || y == bp || op == i || op == bp) {
+                    rescan_row<M>(sh, y);
+                } else {
+                    float bv = sh.bestv[y];
+                    int b2 = op;
+                    const int c1 = i < bp ? i : bp, c2 = i < bp ? bp : i;
+                    const float g1 = c1 == i ? gi : gb, g2 = c2 == i ? gi : gb;
+                    if (g1 > bv || (g1 == bv && c1 < b2)) { bv = g1; b2 = c1; }
+                    if (g2 > bv || (g2 == bv && c2 < b2)) { bv = g2; b2 = c2; }
+                    sh.bestv[y] = bv;
+                    sh.bestp[y] = b2;
+                }
+            }
+            ls_barrier<NT>();                        // row bests complete
+        }
+    }
+}
+
+// Steps 1-4 for one block (M <= 32).  `key` holds this lane's keys (any
+// assignment of the block's entries to positions; padding positions hold
+// Key::sentinel()), `a` the block's |W| (row stride M+1, shared memory).
+// Returns false when the block could not be made feasible (never expected,
+// see the repair proof); the final row bitmasks are in sh.rowbits.
+template <int M, typename Key>
+__device__ bool round_block_warp(Key (&key)[WarpRound<M>::R], const float* a, RoundShared<M>& sh, int N,
+                                 int sweeps, int lane) {
+    constexpr int R = WarpRound<M>::R;
+    warp_bitonic_sort<R>(key, lane);
+    keys_to_order<M>(key, sh, lane);
+    __syncwarp();
+    if (!greedy_and_repair<M, WarpRound<M>::EP>(a, sh, N, lane)) return false;
+    if (sweeps <= 0) return true;
+    __syncwarp();
+    local_search<M>(a, sh, sweeps, lane);
+    return true;
+}
+
+// Row bitmasks of one block into the packed mask (M >= 8: whole bytes,
+// halves or words; M = 4: OR into a zeroed mask, two blocks share a byte).
+template <int M>
+__device__ __forceinline__ void write_mask_rows(uint32_t* mask, int64_t wpr, int64_t r0, int64_t c0,
+                                                const typename WarpRound<M>::Bits* rowbits, bool ok, int lane,
+                                                int nthreads = 32) {
+    for (int r = lane; r < M; r += nthreads) {
+        const unsigned long long bits = ok ? static_cast<unsigned long long>(rowbits[r]) : 0ull;
+        uint32_t* row = mask + (r0 + r) * wpr;
+        if constexpr (M == 64) {
+            row[c0 / 32] = static_cast<uint32_t>(bits);
+            row[c0 / 32 + 1] = static_cast<uint32_t>(bits >> 32);
+        } else if constexpr (M == 32) {
+            row[c0 / 32] = static_cast<uint32_t>(bits);
+        } else if constexpr (M == 16) {
+            reinterpret_cast<uint16_t*>(row)[c0 / 16] = static_cast<uint16_t>(bits);
+        } else if constexpr (M == 8) {
+            reinterpret_cast<uint8_t*>(row)[c0 / 8] = static_cast<uint8_t>(bits);
+        } else {
+            if (bits) atomicOr(&row[c0 / 32], static_cast<uint32_t>(bits) << (c0 % 32));
+        }
+    }
+}
+
+}  // namespace tsenor
+
+namespace tsenor {
+
+// Rounding of a given plan, one warp per block (M <= 32).  Entry e = r*32 + lane
+// of the block (row-major flat index) goes to this lane's register r, so the
+// loads of plan and W are coalesced along block rows.
+template <int M>
+struct RoundWarpSmem {
+    float a[M * (M + 1)];           // |W|, row stride M+1
+    RoundShared<M> sh;
+};
+
+template <int M, typename T>
+__global__ void __launch_bounds__(128)
+round_warp_kernel(const float* __restrict__ plan, const typename T::storage* __restrict__ W, int64_t cols,
+                  int64_t n_blocks, int N, int sweeps, uint32_t* __restrict__ mask, int64_t wpr) {
+    using Key = typename KeyOf<T>::type;
+    constexpr int E = M * M, R = WarpRound<M>::R;
+    extern __shared__ __align__(16) unsigned char round_warp_raw[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    RoundWarpSmem<M>& sm = reinterpret_cast<RoundWarpSmem<M>*>(round_warp_raw)[warp];
+    const int64_t b = int64_t(blockIdx.x) * 4 + warp;
+    if (b >= n_blocks) return;                       // uniform per warp
+    const int64_t nbc = cols / M;
+    const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
+
+    Key key[R];
+    bool ok = true;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int e = r * 32 + lane;
+        if (e < E) {
+            const int i = e / M, j = e % M;
+            const float s = fabsf(plan[(r0 + i) * cols + c0 + j]);
+            const float a = T::load1(W + (r0 + i) * cols + c0 + j);
+            ok = ok && (s <= 3.402823466e38f) && (a <= 3.402823466e38f);
+            sm.a[i * (M + 1) + j] = a;
+            key[r] = Key::make(s, a, e);
+        } else {
+            key[r] = Key::sentinel();
+        }
+    }
+    ok = __all_sync(kFullMask, ok);
+    __syncwarp();
+    if (ok) ok = round_block_warp<M, Key>(key, sm.a, sm.sh, N, sweeps, lane);
+    if (!ok && lane == 0) atomicAdd(&g_block_failures, 1ull);
+    __syncwarp();
+    write_mask_rows<M>(mask, wpr, r0, c0, sm.sh.rowbits, ok, lane);
+}
+
+template <int M>
+constexpr size_t round_warp_smem() { return sizeof(RoundWarpSmem<M>) * 4; }
+
+// Rounding of a given plan for M = 64: one CTA of 4 warps per block.  The
+// 4096 keys are sorted by the whole CTA (32 per thread); greedy, repair and
+// the sweeps run on warp 0; the gain table is filled by all 128 threads.
+template <typename T>
+struct RoundCta64Smem {
+    using Key = typename KeyOf<T>::type;
+    union U {
+        Key xbuf[4096];             // sort exchange between warps
+        RoundShared<64> sh;         // after the sort
+    } u;
+    float a[64 * 65];               // |W|, row stride 65
+    int ok;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(128)
+round_cta64_kernel(const float* __restrict__ plan, const typename T::storage* __restrict__ W, int64_t cols,
+                   int64_t n_blocks, int N, int sweeps, uint32_t* __restrict__ mask, int64_t wpr) {
+    constexpr int M = 64, AS = 65;
+    using Key = typename KeyOf<T>::type;
+    extern __shared__ __align__(16) unsigned char round64_raw[];
+    RoundCta64Smem<T>& sm = *reinterpret_cast<RoundCta64Smem<T>*>(round64_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t b = blockIdx.x;
+    if (b >= n_blocks) return;                       // uniform per CTA
+    const int64_t nbc = cols / M;
+    const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
+
+    Key key[32];
+    bool ok = true;
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+        const int e = r * 128 + tid;
+        const int i = e / M, j = e % M;
+        const float s = fabsf(plan[(r0 + i) * cols + c0 + j]);
+        const float a = T::load1(W + (r0 + i) * cols + c0 + j);
+        ok = ok && (s <= 3.402823466e38f) && (a <= 3.402823466e38f);
+        sm.a[i * AS + j] = a;
+        key[r] = Key::make(s, a, e);
+    }
+    ok = __syncthreads_and(ok);
+    if (ok) {
+        cta_bitonic_sort64(key, sm.u.xbuf, warp, lane);
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < 32; ++r) sm.u.sh.order[tid * 32 + r] = static_cast<uint16_t>(key[r].index());
+        __syncthreads();
+        if (warp == 0) {
+            const bool g = greedy_and_repair<M, 4096>(sm.a, sm.u.sh, N, lane);
+            if (lane == 0) sm.ok = g;
+        }
+        __syncthreads();
+        ok = sm.ok;
+        if (ok && sweeps > 0) {
+            local_search<M>(sm.a, sm.u.sh, sweeps, tid);
+            __syncthreads();
+        }
+    }
+    if (!ok && tid == 0) atomicAdd(&g_block_failures, 1ull);
+    write_mask_rows<M>(mask, wpr, r0, c0, sm.u.sh.rowbits, ok, tid, 128);
+}
+
+}  // namespace tsenor

@@ -8,7 +8,8 @@
 #include "../../include/tsenor.h"
 #include "common.cuh"
 #include "dykstra.cuh"
-#include "rounding.cuh"
+#include "round_warp.cuh"
+#include "fused.cuh"
 #include "objective.cuh"
 
 namespace tsenor {
@@ -64,14 +65,37 @@ cudaError_t launch_round(const float* plan, const void* W, int64_t rows, int64_t
         cudaError_t e = cudaMemsetAsync(mask, 0, size_t(rows) * size_t(wpr) * 4, st);
         if (e != cudaSuccess) return e;
     }
-    constexpr size_t smem = round_smem<M>();
-    cudaError_t e = cudaFuncSetAttribute(round_kernel<M, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(smem));
+    if constexpr (M == 64) {
+        constexpr size_t smem = sizeof(RoundCta64Smem<T>);
+        cudaError_t e = cudaFuncSetAttribute(round_cta64_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(smem));
+        if (e != cudaSuccess) return e;
+        round_cta64_kernel<T><<<dim3(unsigned(nb)), 128, smem, st>>>(
+            plan, static_cast<const typename T::storage*>(W), cols, nb, N, sweeps, mask, wpr);
+    } else {
+        constexpr size_t smem = round_warp_smem<M>();
+        cudaError_t e = cudaFuncSetAttribute(round_warp_kernel<M, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(smem));
+        if (e != cudaSuccess) return e;
+        const int64_t grid = (nb + 3) / 4;
+        round_warp_kernel<M, T><<<dim3(unsigned(grid)), 128, smem, st>>>(
+            plan, static_cast<const typename T::storage*>(W), cols, nb, N, sweeps, mask, wpr);
+    }
+    return cudaGetLastError();
+}
+
+// Whole path in one kernel (M = 32): no workspace.
+template <typename T>
+cudaError_t launch_fused32(const void* W, int64_t rows, int64_t cols, int N, float tau, int iters, int sweeps,
+                           uint32_t* mask, cudaStream_t st) {
+    const int64_t nb = (rows / 32) * (cols / 32);
+    const int64_t wpr = (cols + 31) / 32;
+    constexpr size_t smem = fused32_smem();
+    cudaError_t e = cudaFuncSetAttribute(fused_kernel32<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    constexpr int WP = RoundCfg<M>::WARPS;
-    const int64_t grid = (nb + WP - 1) / WP;
-    round_kernel<M, T><<<dim3(unsigned(grid)), WP * 32, smem, st>>>(
-        plan, static_cast<const typename T::storage*>(W), cols, nb, N, sweeps, mask, wpr);
+    const int64_t grid = (nb + 3) / 4;
+    fused_kernel32<T><<<dim3(unsigned(grid)), 128, smem, st>>>(static_cast<const typename T::storage*>(W), cols, nb,
+                                                                N, tau, iters, sweeps, mask, wpr);
     return cudaGetLastError();
 }
 
@@ -152,6 +176,11 @@ extern "C" tsenor_status tsenor_mask(const void* W, tsenor_dtype dtype, int64_t 
     if (rows == 0 || cols == 0) return TSENOR_OK;
     if (!mask_out || !aligned(mask_out, 8)) return TSENOR_ERR_ARG;
     cudaStream_t st = (cudaStream_t)stream;
+    if (M == 32) {
+        cudaError_t e = dtype == TSENOR_BF16 ? launch_fused32<BF16>(W, rows, cols, N, tau, iters, sweeps, mask_out, st)
+                                             : launch_fused32<F32>(W, rows, cols, N, tau, iters, sweeps, mask_out, st);
+        return e == cudaSuccess ? TSENOR_OK : cuda_fail(e, "tsenor_mask launch");
+    }
     float* plan = nullptr;
     cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&plan), size_t(rows) * size_t(cols) * sizeof(float), st);
     if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask workspace");

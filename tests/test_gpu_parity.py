@@ -203,3 +203,14 @@ def test_stream_ordering_on_side_stream():
     bits = block_bits(mask_to_np(m), 256, 32)
     assert (bits.sum(axis=3) == 16).all()
     assert (block_bits(m_ref, 256, 32) == bits).all(axis=(2, 3)).mean() >= 0.5
+
+
+@pytest.mark.parametrize("c", CASES, ids=_ids)
+def test_mask_equals_rounding_of_exported_plan(c):
+    """tsenor_mask (fused for M = 32) == tsenor_round(tsenor_plan(W)), bit for bit."""
+    M, N, dtype, rows, cols, tau, iters, sweeps, dist = c
+    stor, W = _matrix(c, seed=1)
+    Wd = to_device(stor, dtype)
+    m1 = tsl.tsenor_mask(Wd, N, M, tau, iters, sweeps)
+    m2 = tsl.tsenor_round(tsl.tsenor_plan(Wd, N, M, tau, iters), Wd, N, M, sweeps)
+    assert torch.equal(m1, m2)
