@@ -1,8 +1,12 @@
-// The whole hot path for one block in one warp (M = 32): Dykstra plan kept in
-// registers, sort keys formed from it directly, rounding, packed mask.  No
-// plan ever reaches device memory.  The keys are bit-identical to what the
-// plan kernel writes (same arithmetic), so the result equals rounding the
-// exported plan.
+// The whole hot path in one kernel (M = 16, 32, 64): Dykstra, sort keys from
+// the final state, rounding, packed mask.  No plan ever reaches device
+// memory.  The keys are bit-identical to what the plan kernel writes (same
+// arithmetic), so the result equals rounding the exported plan.
+//  - M = 32: one warp per block; keys straight from the registers.
+//  - M = 16: one warp solves four blocks (8 threads each), writes their plans
+//    to shared memory and rounds them one after another.
+//  - M = 64: one CTA of 4 warps per block; the CTA sorts, warp 0 runs the
+//    greedy and the repair, all 128 threads the local search.
 #pragma once
 
 #include "dykstra.cuh"
@@ -49,6 +53,106 @@ fused_kernel32(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
 
 constexpr size_t fused32_smem() {
     return sizeof(float) * TileCfg<32>::BPC * 32 * 33 + sizeof(RoundShared<32>) * TileCfg<32>::BPC;
+}
+
+// M = 16: a warp holds 4 blocks of 8 threads each.
+template <typename T>
+__global__ void __launch_bounds__(128)
+fused_kernel16(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
+               int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr) {
+    constexpr int M = 16, TS = M + 1, E = M * M;
+    using C = TileCfg<M>;
+    using Key = typename KeyOf<T>::type;
+    constexpr int BPW = C::BPW, R = WarpRound<M>::R;
+    static_assert(C::TPB == 8 && BPW == 4 && C::BPC == 16, "four blocks per warp");
+    extern __shared__ float fused_smem[];
+    float* atiles = fused_smem;                               // [BPC][M * TS] |W|
+    float* ptiles = atiles + C::BPC * M * TS;                 // [BPC][M * M]  plan
+    RoundShared<M>* shs = reinterpret_cast<RoundShared<M>*>(ptiles + C::BPC * E);   // one per warp
+    int* flags = reinterpret_cast<int*>(shs + 4);             // [BPC] finite
+    const TileThread<M> th;
+    float* tile = atiles + th.blk * M * TS;
+    const int64_t b = int64_t(blockIdx.x) * C::BPC + th.blk;
+    const bool active = b < n_blocks;
+    const int64_t nbc = cols / M;
+    const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
+
+    float y[C::P][C::Q];
+    const bool finite = dykstra_tile_solve<M, T, TS>(W, cols, r0, c0, active, N, tau, iters, tile, nullptr, th, y);
+    float* ptile = ptiles + th.blk * E;
+#pragma unroll
+    for (int k = 0; k < C::P; ++k)
+#pragma unroll
+        for (int c = 0; c < C::Q; ++c) ptile[th.row(k) * M + th.col(c)] = plan_value(y[k][c]);
+    if (th.t == 0) flags[th.blk] = finite;
+    __syncwarp();
+
+    const int lane = th.lane, warp = th.warp;
+    for (int s = 0; s < BPW; ++s) {
+        const int slot = warp * BPW + s;
+        const int64_t bb = int64_t(blockIdx.x) * C::BPC + slot;
+        if (bb >= n_blocks) break;                           // uniform over the warp
+        const int64_t rr = (bb / nbc) * M, cc = (bb % nbc) * M;
+        const float* at = atiles + slot * M * TS;
+        const float* pt = ptiles + slot * E;
+        Key key[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int e = r * 32 + lane;
+            key[r] = Key::make(pt[e], at[(e / M) * TS + (e % M)], e);
+        }
+        bool ok = flags[slot] != 0;
+        if (ok) ok = round_block_warp<M, Key>(key, at, shs[warp], N, sweeps, lane);
+        if (!ok && lane == 0) atomicAdd(&g_block_failures, 1ull);
+        __syncwarp();
+        write_mask_rows<M>(mask, wpr, rr, cc, shs[warp].rowbits, ok, lane);
+        __syncwarp();
+    }
+}
+
+constexpr size_t fused16_smem() {
+    return sizeof(float) * 16 * (16 * 17 + 16 * 16) + sizeof(RoundShared<16>) * 4 + sizeof(int) * 16;
+}
+
+// M = 64: one CTA of 4 warps per block.
+template <typename T>
+struct Fused64Smem {
+    RoundCta64Work<typename KeyOf<T>::type> u;
+    float a[64 * 65];                                   // |W|, row stride 65
+    float colbuf[2 * 4 * 32 * TileCfg<64>::CO];         // cross-warp column sums
+    int ok;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(128)
+fused_kernel64(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
+               int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr) {
+    constexpr int M = 64, TS = M + 1;
+    using C = TileCfg<M>;
+    using Key = typename KeyOf<T>::type;
+    static_assert(C::TPB == 128 && C::BPC == 1, "one block per CTA");
+    extern __shared__ __align__(16) unsigned char fused64_raw[];
+    Fused64Smem<T>& sm = *reinterpret_cast<Fused64Smem<T>*>(fused64_raw);
+    const TileThread<M> th;
+    const int64_t b = blockIdx.x;
+    if (b >= n_blocks) return;                         // uniform per CTA
+    const int64_t nbc = cols / M;
+    const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
+
+    float y[C::P][C::Q];
+    const bool finite = dykstra_tile_solve<M, T, TS>(W, cols, r0, c0, true, N, tau, iters, sm.a, sm.colbuf, th, y);
+    Key key[C::P * C::Q];
+#pragma unroll
+    for (int k = 0; k < C::P; ++k)
+#pragma unroll
+        for (int c = 0; c < C::Q; ++c) {
+            const int row = th.row(k), col = th.col(c);
+            key[k * C::Q + c] = Key::make(plan_value(y[k][c]), sm.a[row * TS + col], row * M + col);
+        }
+    bool ok = finite;                                   // uniform over the CTA
+    if (ok) ok = round_block_cta64(key, sm.a, sm.u, &sm.ok, N, sweeps, th.tid);
+    if (!ok && th.tid == 0) atomicAdd(&g_block_failures, 1ull);
+    write_mask_rows<M>(mask, wpr, r0, c0, sm.u.sh.rowbits, ok, th.tid, 128);
 }
 
 }  // namespace tsenor

@@ -576,13 +576,41 @@ constexpr size_t round_warp_smem() { return sizeof(RoundWarpSmem<M>) * 4; }
 // Rounding of a given plan for M = 64: one CTA of 4 warps per block.  The
 // 4096 keys are sorted by the whole CTA (32 per thread); greedy, repair and
 // the sweeps run on warp 0; the gain table is filled by all 128 threads.
+template <typename Key>
+union RoundCta64Work {
+    Key xbuf[4096];                 // sort exchange between warps
+    RoundShared<64> sh;             // after the sort
+};
+
+// Steps 1-4 for one M = 64 block by a CTA of 4 warps (every thread calls it,
+// `ok` uniform over the CTA).  `key`: this thread's 32 keys; `a`: |W| with row
+// stride 65.  The final row bitmasks are in work.sh.rowbits.
+template <typename Key>
+__device__ bool round_block_cta64(Key (&key)[32], const float* a, RoundCta64Work<Key>& work, int* okflag, int N,
+                                  int sweeps, int tid) {
+    constexpr int M = 64;
+    const int lane = tid & 31, warp = tid >> 5;
+    cta_bitonic_sort64(key, work.xbuf, warp, lane);
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < 32; ++r) work.sh.order[tid * 32 + r] = static_cast<uint16_t>(key[r].index());
+    __syncthreads();
+    if (warp == 0) {
+        const bool g = greedy_and_repair<M, 4096>(a, work.sh, N, lane);
+        if (lane == 0) *okflag = g;
+    }
+    __syncthreads();
+    const bool ok = *okflag;
+    if (ok && sweeps > 0) {
+        local_search<M>(a, work.sh, sweeps, tid);
+        __syncthreads();
+    }
+    return ok;
+}
+
 template <typename T>
 struct RoundCta64Smem {
-    using Key = typename KeyOf<T>::type;
-    union U {
-        Key xbuf[4096];             // sort exchange between warps
-        RoundShared<64> sh;         // after the sort
-    } u;
+    RoundCta64Work<typename KeyOf<T>::type> u;
     float a[64 * 65];               // |W|, row stride 65
     int ok;
 };
@@ -595,7 +623,7 @@ round_cta64_kernel(const float* __restrict__ plan, const typename T::storage* __
     using Key = typename KeyOf<T>::type;
     extern __shared__ __align__(16) unsigned char round64_raw[];
     RoundCta64Smem<T>& sm = *reinterpret_cast<RoundCta64Smem<T>*>(round64_raw);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const int64_t b = blockIdx.x;
     if (b >= n_blocks) return;                       // uniform per CTA
     const int64_t nbc = cols / M;
@@ -614,23 +642,7 @@ round_cta64_kernel(const float* __restrict__ plan, const typename T::storage* __
         key[r] = Key::make(s, a, e);
     }
     ok = __syncthreads_and(ok);
-    if (ok) {
-        cta_bitonic_sort64(key, sm.u.xbuf, warp, lane);
-        __syncthreads();
-#pragma unroll
-        for (int r = 0; r < 32; ++r) sm.u.sh.order[tid * 32 + r] = static_cast<uint16_t>(key[r].index());
-        __syncthreads();
-        if (warp == 0) {
-            const bool g = greedy_and_repair<M, 4096>(sm.a, sm.u.sh, N, lane);
-            if (lane == 0) sm.ok = g;
-        }
-        __syncthreads();
-        ok = sm.ok;
-        if (ok && sweeps > 0) {
-            local_search<M>(sm.a, sm.u.sh, sweeps, tid);
-            __syncthreads();
-        }
-    }
+    if (ok) ok = round_block_cta64(key, sm.a, sm.u, &sm.ok, N, sweeps, tid);
     if (!ok && tid == 0) atomicAdd(&g_block_failures, 1ull);
     write_mask_rows<M>(mask, wpr, r0, c0, sm.u.sh.rowbits, ok, tid, 128);
 }

@@ -84,19 +84,47 @@ cudaError_t launch_round(const float* plan, const void* W, int64_t rows, int64_t
     return cudaGetLastError();
 }
 
-// Whole path in one kernel (M = 32): no workspace.
-template <typename T>
-cudaError_t launch_fused32(const void* W, int64_t rows, int64_t cols, int N, float tau, int iters, int sweeps,
-                           uint32_t* mask, cudaStream_t st) {
-    const int64_t nb = (rows / 32) * (cols / 32);
+// Whole path in one kernel (M = 16, 32, 64): no workspace.
+template <int M, typename T>
+cudaError_t launch_fused(const void* W, int64_t rows, int64_t cols, int N, float tau, int iters, int sweeps,
+                         uint32_t* mask, cudaStream_t st) {
+    const int64_t nb = (rows / M) * (cols / M);
     const int64_t wpr = (cols + 31) / 32;
-    constexpr size_t smem = fused32_smem();
-    cudaError_t e = cudaFuncSetAttribute(fused_kernel32<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    const int64_t grid = (nb + 3) / 4;
-    fused_kernel32<T><<<dim3(unsigned(grid)), 128, smem, st>>>(static_cast<const typename T::storage*>(W), cols, nb,
-                                                                N, tau, iters, sweeps, mask, wpr);
+    const auto* w = static_cast<const typename T::storage*>(W);
+    cudaError_t e = cudaSuccess;
+    if constexpr (M == 32) {
+        constexpr size_t smem = fused32_smem();
+        e = cudaFuncSetAttribute(fused_kernel32<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        fused_kernel32<T><<<dim3(unsigned((nb + 3) / 4)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps, mask,
+                                                                          wpr);
+    } else if constexpr (M == 16) {
+        if (cols % 32) {
+            e = cudaMemsetAsync(mask, 0, size_t(rows) * size_t(wpr) * 4, st);   // padding bits
+            if (e != cudaSuccess) return e;
+        }
+        constexpr size_t smem = fused16_smem();
+        e = cudaFuncSetAttribute(fused_kernel16<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        fused_kernel16<T><<<dim3(unsigned((nb + 15) / 16)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps,
+                                                                            mask, wpr);
+    } else {
+        constexpr size_t smem = sizeof(Fused64Smem<T>);
+        e = cudaFuncSetAttribute(fused_kernel64<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        fused_kernel64<T><<<dim3(unsigned(nb)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps, mask, wpr);
+    }
     return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t dispatch_fused(int M, const void* W, int64_t rows, int64_t cols, int N, float tau, int iters, int sweeps,
+                           uint32_t* mask, cudaStream_t st) {
+    switch (M) {
+        case 16: return launch_fused<16, T>(W, rows, cols, N, tau, iters, sweeps, mask, st);
+        case 32: return launch_fused<32, T>(W, rows, cols, N, tau, iters, sweeps, mask, st);
+        default: return launch_fused<64, T>(W, rows, cols, N, tau, iters, sweeps, mask, st);
+    }
 }
 
 template <typename T>
@@ -176,9 +204,9 @@ extern "C" tsenor_status tsenor_mask(const void* W, tsenor_dtype dtype, int64_t 
     if (rows == 0 || cols == 0) return TSENOR_OK;
     if (!mask_out || !aligned(mask_out, 8)) return TSENOR_ERR_ARG;
     cudaStream_t st = (cudaStream_t)stream;
-    if (M == 32) {
-        cudaError_t e = dtype == TSENOR_BF16 ? launch_fused32<BF16>(W, rows, cols, N, tau, iters, sweeps, mask_out, st)
-                                             : launch_fused32<F32>(W, rows, cols, N, tau, iters, sweeps, mask_out, st);
+    if (M >= 16) {
+        cudaError_t e = dtype == TSENOR_BF16 ? dispatch_fused<BF16>(M, W, rows, cols, N, tau, iters, sweeps, mask_out, st)
+                                             : dispatch_fused<F32>(M, W, rows, cols, N, tau, iters, sweeps, mask_out, st);
         return e == cudaSuccess ? TSENOR_OK : cuda_fail(e, "tsenor_mask launch");
     }
     float* plan = nullptr;
