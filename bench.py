@@ -140,6 +140,27 @@ class ClockSampler:
                 "power_w_max": max((float(p[3]) for p in use if p[3].replace(".", "").isdigit()), default=None)}
 
 
+def rank_seed(w, rank: int) -> int:
+    """Each rank solves its own matrix of the workload's shape (weak scaling)."""
+    return w.seed + rank
+
+
+def max_over_ranks(value: float, device, world: int) -> float:
+    """Max of a per-rank scalar over all ranks (the step time of the slowest rank)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_gparams(params_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: parameters solved by all ranks over the slowest rank's time."""
+    return params_per_rank * world / (max_ms / 1e3) / 1e9
+
+
 def to_device(storage, dtype, device):
     import torch
     if dtype == "bf16":
@@ -248,7 +269,7 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
     w = synth.WORKLOADS[args.workload]
-    storage, vals = synth.workload_matrix(w, seed=w.seed + rank)
+    storage, vals = synth.workload_matrix(w, seed=rank_seed(w, rank))
     Wd = to_device(storage, w.dtype, dev)
     wpr = (w.cols + 31) // 32
     mask = torch.empty((w.rows, wpr), dtype=torch.int32, device=dev)
@@ -283,10 +304,7 @@ def main(argv=None):
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     mean_ms = sum(step_ms) / len(step_ms)
-    t_max = torch.tensor([mean_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    mean_ms_max = float(t_max.item())
+    mean_ms_max = max_over_ranks(mean_ms, dev, world)
     clocks = sampler.stop()
     gpu_mask = mask.cpu().numpy().view(np.uint32)
 
@@ -323,13 +341,10 @@ def main(argv=None):
             e2e_ev.append((a, b))
     torch.cuda.synchronize(dev)
     e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in e2e_ev)
-    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev, world)
 
     params = w.rows * w.cols
-    value = params * world / (mean_ms_max / 1e3) / 1e9
+    value = aggregate_gparams(params, world, mean_ms_max)
     ops_per_param = w.iters * (1.0 + 2.0 / w.M)
     peak = mufu_peak_tops(SM_MAX_MHZ_FALLBACK)
     if w.M == 32:
@@ -361,7 +376,7 @@ def main(argv=None):
                      "kernel_ms": kernel_ms},
         "breakdown_ms": {"dykstra_plan_kernel_alone": plan_ms, "rest_of_step": round_ms,
                          "dykstra_frac_of_peak": params * ops_per_param / (plan_ms / 1e3) / 1e12 / peak},
-        "e2e": {"value": params * world / (e2e_ms / 1e3) / 1e9, "unit": "Gparams/s",
+        "e2e": {"value": aggregate_gparams(params, world, e2e_ms), "unit": "Gparams/s",
                 "h2d_bytes_per_step": int(storage.nbytes), "d2h_bytes_per_step": int(host_mask.numel() * 4),
                 "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,

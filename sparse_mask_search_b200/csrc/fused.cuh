@@ -9,13 +9,17 @@
 //    greedy and the repair, all 128 threads the local search.
 #pragma once
 
+#include <type_traits>
+
 #include "dykstra.cuh"
 #include "round_warp.cuh"
 
 namespace tsenor {
 
+// bf16: registers capped for 5 CTAs (20 warps) per SM (5.00 ms against 5.03 ms
+// uncapped on the 4096x11008 16:32 workload); the fp32 key needs more.
 template <typename T>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, std::is_same<T, BF16>::value ? 5 : 4)
 fused_kernel32(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
                int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr) {
     constexpr int M = 32;
