@@ -32,6 +32,7 @@ import numpy as np  # noqa: E402
 import synth  # noqa: E402
 
 DEFAULT_WORKLOAD = "w4096x11008_bf16_t3_16of32"
+STACK = "stack7b"                  # 32 layers x 7 matrices, 4:8, one pass = one step
 SM_COUNT = 148
 MUFU_PER_CLK_PER_SM = 16          # ex2 / lg2 / rcp results per clock per SM
 SM_MAX_MHZ_FALLBACK = 1965.0
@@ -44,7 +45,8 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=60)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS) + [STACK])
+    p.add_argument("--layers", type=int, default=synth.STACK_7B_LAYERS, help="layers of the 7B stack")
     p.add_argument("--cpu-seconds", type=float, default=15.0,
                    help="target CPU time of the bounded oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -216,8 +218,16 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     import oracle
-    w = synth.WORKLOADS[args.workload]
-    _, vals = synth.workload_matrix(w)
+    if args.workload == STACK:
+        # a bounded sample of the stack: block-rows of layer 0's first matrix
+        st = synth.STACK_7B_SETTINGS
+        name, r, c = synth.STACK_7B_MATRICES[0]
+        w = synth.Workload(f"stack7b_layer0_{name}", r, c, "bf16", "normal", 0.02, st["N"], st["M"], st["tau"],
+                           st["iters"], st["sweeps"], 0)
+        _, vals = synth.make_matrix(r, c, "bf16", "normal", 0.02, 0)
+    else:
+        w = synth.WORKLOADS[args.workload]
+        _, vals = synth.workload_matrix(w)
     cores = oracle.threads_used(0)
     M = w.M
     t = time.perf_counter()
@@ -248,6 +258,76 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------------------- 7B stack
+
+def run_stack(args, rank, world):
+    """One step = tsenor_mask over every matrix of the 7B-shaped stack, layer by layer."""
+    import torch
+    import sparse_mask_search_b200 as tsl
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    st = synth.STACK_7B_SETTINGS
+    N, M, tau, iters, sweeps = st["N"], st["M"], st["tau"], st["iters"], st["sweeps"]
+    mats = []
+    t_gen = time.perf_counter()
+    for layer in range(rank * args.layers, (rank + 1) * args.layers):      # ranks split whole layers
+        for name, bits, _ in synth.stack_7b_layer(layer):
+            Wd = to_device(bits, "bf16", dev)
+            mats.append((layer, name, Wd, torch.empty((Wd.shape[0], (Wd.shape[1] + 31) // 32),
+                                                     dtype=torch.int32, device=dev)))
+    t_gen = time.perf_counter() - t_gen
+    stream = torch.cuda.current_stream(dev)
+    params = sum(Wd.numel() for _, _, Wd, _ in mats)
+
+    def one_pass():
+        for _, _, Wd, out in mats:
+            tsl.tsenor_mask(Wd, N, M, tau, iters, sweeps, out=out, stream=stream)
+
+    for _ in range(max(1, args.warmup)):
+        for _, _, Wd, out in mats[:7]:
+            tsl.tsenor_mask(Wd, N, M, tau, iters, sweeps, out=out, stream=stream)
+    torch.cuda.synchronize(dev)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    time.sleep(0.3)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.mark_start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in ev:
+        a.record(stream)
+        one_pass()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.mark_end()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    ms_max = max_over_ranks(ms, dev, world)
+    clocks = sampler.stop()
+    tsl.tsenor_error_count()
+    line = {
+        "metric": "transposable N:M mask Gparams/s at 1 B200 (% of roofline); mean gap to exact opt",
+        "value": aggregate_gparams(params, world, ms_max), "unit": "Gparams/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"stack7b_{args.layers}x7_bf16_4of8", "layers_per_rank": args.layers,
+                   "matrices_per_rank": len(mats), "params_per_rank": params, "N": N, "M": M, "tau": tau,
+                   "iters": iters, "sweeps": sweeps,
+                   "l2": "inputs larger than L2 (13 GB per pass, each matrix read once per pass)",
+                   "total_wall_s_per_pass": ms_max / 1e3, "host_generation_s": t_gen},
+        "roofline": {"bound": "alu", "achieved": params * iters * (1 + 2.0 / M) / (ms / 1e3) / 1e12,
+                     "peak": mufu_peak_tops(SM_MAX_MHZ_FALLBACK), "unit": "TOP/s",
+                     "frac": params * iters * (1 + 2.0 / M) / (ms / 1e3) / 1e12 / mufu_peak_tops(SM_MAX_MHZ_FALLBACK),
+                     "traffic": None, "kernel": "whole pass (dykstra_thread_kernel<8> + round_warp_kernel<8>)"},
+        "gpu_launches": 2 * len(mats) * args.steps,
+        "clocks": clocks, "cpu_baseline": None,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # --------------------------------------------------------------------------- GPU leg
 
 def main(argv=None):
@@ -257,6 +337,18 @@ def main(argv=None):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return 0
+    if args.workload == STACK:
+        if world > 1:
+            import torch
+            import torch.distributed as dist
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        run_stack(args, rank, world)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
         return 0
 
     import torch
@@ -347,15 +439,14 @@ def main(argv=None):
     value = aggregate_gparams(params, world, mean_ms_max)
     ops_per_param = w.iters * (1.0 + 2.0 / w.M)
     peak = mufu_peak_tops(SM_MAX_MHZ_FALLBACK)
-    if w.M == 32:
-        # tsenor_mask is one fused kernel for M = 32: the dominant kernel is the
-        # whole step; the plan-only kernel gives the Dykstra phase alone
-        kernel_key = f"fused_kernel32<{w.dtype}>"
+    if w.M >= 16:
+        # tsenor_mask is one fused kernel for M = 16, 32, 64: the dominant kernel
+        # is the whole step; the plan-only kernel gives the Dykstra phase alone
+        kernel_key = f"fused_kernel{w.M}<{w.dtype}>"
         kernel_ms = mean_ms
         launches_per_step = 1
     else:
-        kernel_key = (f"dykstra_tile_kernel<{w.M},{w.dtype}>" if w.M >= 16
-                      else f"dykstra_thread_kernel<{w.M},{w.dtype}>")
+        kernel_key = f"dykstra_thread_kernel<{w.M},{w.dtype}>"
         kernel_ms = plan_ms
         launches_per_step = 2
     achieved = params * ops_per_param / (kernel_ms / 1e3) / 1e12

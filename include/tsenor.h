@@ -22,7 +22,9 @@
  *    owned by the caller; the library keeps none of them after the call.
  *    W and the plan must be 16-byte aligned; the mask 8-byte aligned.
  *  - W is row-major, rows x cols, of the element type `dtype`; only |W| is
- *    used.  rows and cols must be multiples of M (the review leaves other
+ *    used, so any matrix of importance scores (for example |W_ij| times the
+ *    norm of input feature j, as layer-wise pruning methods use) can be
+ *    passed in its place.  rows and cols must be multiples of M (the review leaves other
  *    shapes open, "Assumptions & free parameters"); rows == 0 or cols == 0
  *    is a valid empty call that does nothing.
  *  - Supported M: 4, 8, 16, 32, 64.  1 <= N <= M.  tau > 0 and finite,
@@ -114,6 +116,41 @@ tsenor_status tsenor_objective(const void* W, tsenor_dtype dtype, int64_t rows, 
  * move) since the previous call, and resets the counter.
  */
 tsenor_status tsenor_error_count(tsenor_stream_t stream, int64_t* count_out);
+
+/*
+ * tsenor_mask with the monotonicity safeguard of the review's "Assumptions &
+ * free parameters" (Assumption 1 of Theorem 1; referee comment 2): inside an
+ * outer loop (an ADMM mask update) the new mask must not lower the block
+ * objective below the previous mask's.  Per block: the new mask is computed
+ * as by tsenor_mask; when prev_mask's block is a valid N:M block whose kept
+ * sum of |W| is strictly larger, prev_mask's block is written instead.  Both
+ * sums are taken in fp64 in row-major order within the block.
+ *   prev_mask: rows x words_per_row uint32 (device), same layout as mask_out;
+ *              it may not alias mask_out.
+ *   kept_out:  optional device counter (may be NULL); the number of blocks that
+ *              kept prev_mask is ADDED to it.
+ */
+tsenor_status tsenor_mask_safeguard(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
+                                    int N, int M, float tau, int iters, int sweeps,
+                                    const uint32_t* prev_mask, uint32_t* mask_out,
+                                    unsigned long long* kept_out, tsenor_stream_t stream);
+
+/*
+ * tsenor_mask for shapes that are not multiples of M.  The review leaves
+ * such shapes open ("Assumptions & free parameters": the partition into MxM
+ * blocks "with no remainder or with padding"); this entry point takes the
+ * padding reading: W is extended with zeros to ceil(rows/M)*M x
+ * ceil(cols/M)*M, every block of the extended matrix is solved, and mask_out
+ * receives the rows x cols part (words_per_row = ceil(cols/32), bits past
+ * cols are 0).  In a full block every row and column keeps exactly N entries;
+ * in an edge block a real row or column keeps at most N.
+ *   W: rows x cols, row-major, no alignment requirement.
+ * Uses stream-ordered workspaces (cudaMallocAsync / cudaFreeAsync) for the
+ * padded copy of W and its mask.
+ */
+tsenor_status tsenor_mask_padded(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
+                                 int N, int M, float tau, int iters, int sweeps,
+                                 uint32_t* mask_out, tsenor_stream_t stream);
 
 /* Static description of a status code. */
 const char* tsenor_status_string(int status);

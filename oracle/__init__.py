@@ -42,6 +42,8 @@ def lib():
         L.oracle_objective.argtypes = [p, p, i64, i64, i32, i32, p]
         L.oracle_opt.argtypes = [p, i64, i64, i32, i32, p, p, i32]
         L.oracle_threads_used.argtypes = [i32]
+        L.oracle_safeguard.argtypes = [p, p, p, i64, i64, i32, i32, p]
+        L.oracle_safeguard.restype = i64
         _lib = L
     return _lib
 
@@ -143,6 +145,19 @@ def opt(W, N, M, threads=0, want_mask=False):
     m = np.zeros((rows, words_per_row(cols)), dtype=np.uint32) if want_mask else None
     _check(lib().oracle_opt(_ptr(W), rows, cols, N, M, _ptr(out), _ptr(m), threads))
     return out, m
+
+
+def safeguard(W, prev_mask, new_mask, N, M):
+    """Per block keep the previous mask if valid and strictly heavier; returns (mask, kept blocks)."""
+    W = _f32(W)
+    rows, cols = W.shape
+    prev = np.ascontiguousarray(prev_mask, dtype=np.uint32)
+    new = np.ascontiguousarray(new_mask, dtype=np.uint32)
+    out = np.empty_like(new)
+    kept = lib().oracle_safeguard(_ptr(W), _ptr(prev), _ptr(new), rows, cols, N, M, _ptr(out))
+    if kept < 0:
+        raise ValueError("oracle rejected the arguments")
+    return out, int(kept)
 
 
 def unpack(mask_words, cols):

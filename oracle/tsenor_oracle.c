@@ -571,3 +571,56 @@ int oracle_opt(const float* W, int64_t rows, int64_t cols, int N, int M, double*
     if (bits) { pack_bits(bits, rows, cols, mask_out); free(bits); }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Monotonicity safeguard ("Assumptions & free parameters", Assumption 1 of
+ * Theorem 1; referee comment 2): per block, keep the previous mask when it is
+ * a valid N:M block whose kept mass exceeds the new mask's.  Kept mass is
+ * summed in fp64 over the block in row-major order.  out may alias new_mask.
+ * Returns the number of blocks that kept the previous mask. */
+static double block_mass(const float* W, const uint32_t* mask, int64_t cols, int M, int64_t br, int64_t bc,
+                         int N, int* valid) {
+    const int64_t wpr = (cols + 31) / 32;
+    double obj = 0.0;
+    int cc[64];
+    for (int j = 0; j < M; ++j) cc[j] = 0;
+    *valid = 1;
+    for (int i = 0; i < M; ++i) {
+        int rcnt = 0;
+        for (int j = 0; j < M; ++j) {
+            const int64_t row = br * M + i, col = bc * M + j;
+            if ((mask[row * wpr + col / 32] >> (col % 32)) & 1u) {
+                obj += (double)fabsf(W[row * cols + col]);
+                rcnt++; cc[j]++;
+            }
+        }
+        if (rcnt != N) *valid = 0;
+    }
+    for (int j = 0; j < M; ++j) if (cc[j] != N) *valid = 0;
+    return obj;
+}
+
+int64_t oracle_safeguard(const float* W, const uint32_t* prev_mask, const uint32_t* new_mask, int64_t rows,
+                         int64_t cols, int N, int M, uint32_t* out) {
+    if (check_args(rows, cols, N, M)) return -1;
+    const int64_t nbr = rows / M, nbc = cols / M, wpr = (cols + 31) / 32;
+    if (out != new_mask) memcpy(out, new_mask, sizeof(uint32_t) * (size_t)(rows * wpr));
+    int64_t kept = 0;
+    for (int64_t br = 0; br < nbr; ++br)
+        for (int64_t bc = 0; bc < nbc; ++bc) {
+            int vp = 0, vn = 0;
+            const double op = block_mass(W, prev_mask, cols, M, br, bc, N, &vp);
+            const double on = block_mass(W, new_mask, cols, M, br, bc, N, &vn);
+            if (vp && op > on) {
+                kept++;
+                for (int i = 0; i < M; ++i)
+                    for (int j = 0; j < M; ++j) {
+                        const int64_t row = br * M + i, col = bc * M + j;
+                        const uint32_t bit = 1u << (col % 32);
+                        uint32_t* w = out + row * wpr + col / 32;
+                        if ((prev_mask[row * wpr + col / 32] >> (col % 32)) & 1u) *w |= bit; else *w &= ~bit;
+                    }
+            }
+        }
+    return kept;
+}

@@ -17,7 +17,8 @@ STATUS = {0: "TSENOR_OK", -1: "TSENOR_ERR_ARG", -2: "TSENOR_ERR_SHAPE", -3: "TSE
           -4: "TSENOR_ERR_CUDA", -5: "TSENOR_ERR_TOO_LARGE"}
 NOALLOC_MAX_PARAMS = 16 * 1024 * 1024
 EXPORTS = ("tsenor_mask", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
-           "tsenor_status_string", "tsenor_last_error", "tsenor_mask_noalloc")
+           "tsenor_status_string", "tsenor_last_error", "tsenor_mask_noalloc", "tsenor_mask_safeguard",
+           "tsenor_mask_padded")
 
 _lib = None
 
@@ -40,6 +41,8 @@ def lib() -> C.CDLL:
         L.tsenor_mask.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p]
         L.tsenor_mask_noalloc.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p]
         L.tsenor_plan.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, p, p]
+        L.tsenor_mask_padded.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p]
+        L.tsenor_mask_safeguard.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p, p, p]
         L.tsenor_round.argtypes = [p, p, i32, i64, i64, i32, i32, i32, p, p]
         L.tsenor_objective.argtypes = [p, i32, i64, i64, p, i32, i32, p, p]
         L.tsenor_error_count.argtypes = [p, C.POINTER(C.c_int64)]
@@ -119,6 +122,36 @@ def tsenor_mask_noalloc(W, N: int, M: int, tau: float, iters: int, sweeps: int, 
     return out
 
 
+def tsenor_mask_safeguard(W, prev_mask, N: int, M: int, tau: float, iters: int, sweeps: int, out=None,
+                          kept=None, stream=None):
+    """tsenor_mask that keeps, per block, prev_mask where it is valid and keeps more |W|.
+
+    ``kept`` (optional int64 CUDA tensor of one element) receives the count of
+    blocks that kept prev_mask (added to its value).
+    """
+    import torch
+    _check_2d_cuda(W, "W")
+    rows, cols = W.shape
+    if out is None:
+        out = torch.empty((rows, words_per_row(cols)), dtype=torch.int32, device=W.device)
+    _check(lib().tsenor_mask_safeguard(W.data_ptr(), _dtype_code(W), rows, cols, N, M, float(tau), iters, sweeps,
+                                       prev_mask.data_ptr(), out.data_ptr(),
+                                       kept.data_ptr() if kept is not None else None, _stream_handle(stream)))
+    return out
+
+
+def tsenor_mask_padded(W, N: int, M: int, tau: float, iters: int, sweeps: int, out=None, stream=None):
+    """tsenor_mask for any shape: W is zero-padded to multiples of M, the mask cropped back."""
+    import torch
+    _check_2d_cuda(W, "W")
+    rows, cols = W.shape
+    if out is None:
+        out = torch.empty((rows, words_per_row(cols)), dtype=torch.int32, device=W.device)
+    _check(lib().tsenor_mask_padded(W.data_ptr(), _dtype_code(W), rows, cols, N, M, float(tau), iters, sweeps,
+                                    out.data_ptr(), _stream_handle(stream)))
+    return out
+
+
 def tsenor_plan(W, N: int, M: int, tau: float, iters: int, out=None, stream=None):
     """Fractional plan S (fp32, same shape as W) after `iters` Dykstra iterations."""
     import torch
@@ -165,5 +198,5 @@ def tsenor_error_count(stream=None) -> int:
     return int(n.value)
 
 
-__all__ = ["tsenor_mask", "tsenor_mask_noalloc", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
+__all__ = ["tsenor_mask", "tsenor_mask_noalloc", "tsenor_mask_safeguard", "tsenor_mask_padded", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
            "TsenorError", "lib", "words_per_row", "EXPORTS", "LIB_PATH"]

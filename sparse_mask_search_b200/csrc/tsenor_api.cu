@@ -220,6 +220,62 @@ extern "C" tsenor_status tsenor_mask(const void* W, tsenor_dtype dtype, int64_t 
     return TSENOR_OK;
 }
 
+extern "C" tsenor_status tsenor_mask_safeguard(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
+                                               int N, int M, float tau, int iters, int sweeps,
+                                               const uint32_t* prev_mask, uint32_t* mask_out,
+                                               unsigned long long* kept_out, tsenor_stream_t stream) {
+    tsenor_status s = check_common(W, dtype, rows, cols, N, M);
+    if (s != TSENOR_OK) return s;
+    if (!solver_params_ok(tau, iters) || sweeps < 0) return TSENOR_ERR_ARG;
+    if (rows == 0 || cols == 0) return TSENOR_OK;
+    if (!prev_mask || !aligned(prev_mask, 8) || prev_mask == mask_out) return TSENOR_ERR_ARG;
+    if (kept_out && !aligned(kept_out, 8)) return TSENOR_ERR_ARG;
+    s = tsenor_mask(W, dtype, rows, cols, N, M, tau, iters, sweeps, mask_out, stream);
+    if (s != TSENOR_OK) return s;
+    cudaError_t e = launch_safeguard(dtype == TSENOR_BF16, W, rows, cols, prev_mask, mask_out, N, M, kept_out,
+                                     (cudaStream_t)stream);
+    return e == cudaSuccess ? TSENOR_OK : cuda_fail(e, "tsenor_mask_safeguard launch");
+}
+
+extern "C" tsenor_status tsenor_mask_padded(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols, int N,
+                                            int M, float tau, int iters, int sweeps, uint32_t* mask_out,
+                                            tsenor_stream_t stream) {
+    if (M != 4 && M != 8 && M != 16 && M != 32 && M != 64) return TSENOR_ERR_UNSUPPORTED_M;
+    if (dtype != TSENOR_F32 && dtype != TSENOR_BF16) return TSENOR_ERR_ARG;
+    if (N < 1 || N > M || !solver_params_ok(tau, iters) || sweeps < 0) return TSENOR_ERR_ARG;
+    if (rows < 0 || cols < 0 || rows > (int64_t(1) << 31) || cols > (int64_t(1) << 31)) return TSENOR_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return TSENOR_OK;
+    if (!W || !mask_out || !aligned(mask_out, 4)) return TSENOR_ERR_ARG;
+    if (rows % M == 0 && cols % M == 0 && aligned(W, 16) && aligned(mask_out, 8))
+        return tsenor_mask(W, dtype, rows, cols, N, M, tau, iters, sweeps, mask_out, stream);
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t es = dtype == TSENOR_BF16 ? 2 : 4;
+    const int64_t rp = (rows + M - 1) / M * M, cp = (cols + M - 1) / M * M;
+    const int64_t wpr = (cols + 31) / 32, wprp = (cp + 31) / 32;
+    void* Wp = nullptr;
+    uint32_t* mp = nullptr;
+    cudaError_t e = cudaMallocAsync(&Wp, size_t(rp) * size_t(cp) * es, st);
+    if (e == cudaSuccess) e = cudaMallocAsync(reinterpret_cast<void**>(&mp), size_t(rp) * size_t(wprp) * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(Wp, 0, size_t(rp) * size_t(cp) * es, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(Wp, size_t(cp) * es, W, size_t(cols) * es, size_t(cols) * es, size_t(rows),
+                              cudaMemcpyDeviceToDevice, st);
+    tsenor_status s = TSENOR_OK;
+    if (e == cudaSuccess) s = tsenor_mask(Wp, dtype, rp, cp, N, M, tau, iters, sweeps, mp, stream);
+    if (e == cudaSuccess && s == TSENOR_OK) {
+        const int64_t n = rows * wpr;
+        crop_mask_kernel<<<unsigned((n + 255) / 256), 256, 0, st>>>(mp, wprp, mask_out, wpr, rows, cols);
+        e = cudaGetLastError();
+    }
+    cudaError_t e2 = Wp ? cudaFreeAsync(Wp, st) : cudaSuccess;
+    cudaError_t e3 = mp ? cudaFreeAsync(mp, st) : cudaSuccess;
+    if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask_padded");
+    if (s != TSENOR_OK) return s;
+    if (e2 != cudaSuccess) return cuda_fail(e2, "tsenor_mask_padded free");
+    if (e3 != cudaSuccess) return cuda_fail(e3, "tsenor_mask_padded free");
+    return TSENOR_OK;
+}
+
 extern "C" tsenor_status tsenor_objective(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
                                           const uint32_t* mask, int N, int M, double* out,
                                           tsenor_stream_t stream) {

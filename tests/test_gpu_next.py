@@ -1,0 +1,81 @@
+"""Extensions beyond the core path, against the oracle:
+  - score matrices in place of W (review: the solver plugs into layer-wise
+    pruning such as Wanda, SparseGPT, ALPS, which hand it importance scores);
+  - the monotonicity safeguard (review: "Assumptions & free parameters",
+    Assumption 1; referee comment 2).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import block_bits, mask_to_np, to_device
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import sparse_mask_search_b200 as tsl  # noqa: E402
+
+
+@pytest.mark.parametrize("M,N", [(8, 4), (16, 8), (32, 16), (64, 32)])
+def test_wanda_style_scores(M, N):
+    rows, cols = 2 * M, 6 * M
+    _, W = synth.make_matrix(rows, cols, "f32", "normal", 0.02, seed=M)
+    xnorm = 0.5 + synth.rng(100 + M).random(cols).astype(np.float32)       # input feature norms
+    scores = (np.abs(W) * xnorm[None, :]).astype(np.float32)
+    m = mask_to_np(tsl.tsenor_mask(to_device(scores, "f32"), N, M, 20.0, 200, 4))
+    m_ref, _, _ = oracle.mask(scores, N, M, 20.0, 200, 4)
+    bg, br = block_bits(m, cols, M), block_bits(m_ref, cols, M)
+    assert (bg.sum(axis=3) == N).all() and (bg.sum(axis=2) == N).all()
+    assert (bg == br).all()
+
+
+@pytest.mark.parametrize("M,N,dtype", [(4, 2, "f32"), (8, 4, "bf16"), (16, 5, "bf16"), (32, 16, "bf16"),
+                                       (64, 32, "bf16")])
+def test_safeguard_matches_oracle(M, N, dtype):
+    rows, cols = 2 * M, 9 * M
+    stor, W = synth.make_matrix(rows, cols, dtype, "t3_outlier_cols", 0.02, seed=7 + M)
+    Wd = to_device(stor, dtype)
+    tau, iters, sweeps = 20.0, 150, 4
+    new = mask_to_np(tsl.tsenor_mask(Wd, N, M, tau, iters, sweeps))
+    opt, best = oracle.opt(W, N, M, want_mask=True)
+    prev_cases = [best, new, np.full_like(new, 0xFFFFFFFF)]
+    for prev in prev_cases:
+        kept = torch.zeros(1, dtype=torch.int64, device="cuda")
+        prev_d = torch.from_numpy(np.ascontiguousarray(prev).view(np.int32)).cuda()
+        out = mask_to_np(tsl.tsenor_mask_safeguard(Wd, prev_d, N, M, tau, iters, sweeps, kept=kept))
+        ref, kept_ref = oracle.safeguard(W, prev, new, N, M)
+        assert (out == ref).all()
+        assert int(kept.item()) == kept_ref
+    # with the optimum as the previous mask the result is optimal everywhere
+    kept = torch.zeros(1, dtype=torch.int64, device="cuda")
+    out = tsl.tsenor_mask_safeguard(Wd, torch.from_numpy(best.view(np.int32)).cuda(), N, M, tau, iters, sweeps,
+                                    kept=kept)
+    np.testing.assert_allclose(tsl.tsenor_objective(Wd, out, N, M).cpu().numpy(), opt, rtol=1e-12)
+
+
+@pytest.mark.parametrize("rows,cols,M,N,dtype", [(100, 70, 32, 16, "bf16"), (50, 37, 8, 4, "f32"),
+                                                 (17, 48, 16, 8, "bf16"), (64, 64, 16, 8, "bf16"),
+                                                 (9, 130, 64, 32, "bf16"), (6, 10, 4, 2, "f32")])
+def test_padded_shapes(rows, cols, M, N, dtype):
+    """Zero-pad to multiples of M, solve, crop (the padding reading of the review's block partition)."""
+    stor, W = synth.make_matrix(rows, cols, dtype, "normal", 0.02, seed=rows + cols)
+    m = mask_to_np(tsl.tsenor_mask_padded(to_device(stor, dtype), N, M, 20.0, 150, 4))
+    rp, cp = -(-rows // M) * M, -(-cols // M) * M
+    Wp = np.zeros((rp, cp), np.float32)
+    Wp[:rows, :cols] = W
+    m_ref_p, _, _ = oracle.mask(Wp, N, M, 20.0, 150, 4)
+    ref_bits = oracle.unpack(m_ref_p, cp)[:rows, :cols]
+    bits = oracle.unpack(m, cols)
+    assert m.shape == (rows, (cols + 31) // 32)
+    assert (oracle.unpack(m, m.shape[1] * 32)[:, cols:] == 0).all()       # padding bits are 0
+    assert (bits == ref_bits).all()
+    # every row / column of a block keeps at most N (exactly N where the block is full)
+    full_r, full_c = rows // M * M, cols // M * M
+    if full_r and full_c:
+        fb = oracle.blocks_view(bits[:full_r, :full_c], M)
+        assert (fb.sum(axis=3) == N).all() and (fb.sum(axis=2) == N).all()
+    for r0 in range(0, rows, M):
+        for c0 in range(0, cols, M):
+            blk = bits[r0:r0 + M, c0:c0 + M]
+            assert (blk.sum(axis=1) <= N).all() and (blk.sum(axis=0) <= N).all()
