@@ -44,6 +44,9 @@ def lib():
         L.oracle_threads_used.argtypes = [i32]
         L.oracle_safeguard.argtypes = [p, p, p, i64, i64, i32, i32, p]
         L.oracle_safeguard.restype = i64
+        L.oracle_block_plan_ext.argtypes = [p, i32, i32, f64, i32, f64, i32, p, p]
+        L.oracle_solve_ext.argtypes = [p, i64, i64, i32, i32, f64, i32, i32, f64, i32, p, p, p, p, i32,
+                                       C.POINTER(Stats)]
         _lib = L
     return _lib
 
@@ -158,6 +161,45 @@ def safeguard(W, prev_mask, new_mask, N, M):
     if kept < 0:
         raise ValueError("oracle rejected the arguments")
     return out, int(kept)
+
+
+def block_plan_ext(a, N, tau, iters, tol=0.0, uv=None):
+    """Plan of one block with warm start / adaptive stopping.
+
+    uv: starting potentials (2M, U then V, nats) or None for a cold start.
+    Returns (S fp64 MxM, final potentials (2M,), iterations run).
+    """
+    a = _f32(np.abs(a))
+    M = a.shape[0]
+    S = np.empty((M, M), dtype=np.float64)
+    warm = uv is not None
+    buf = np.array(uv, dtype=np.float64).copy() if warm else np.zeros(2 * M, dtype=np.float64)
+    t = lib().oracle_block_plan_ext(_ptr(a), N, M, float(tau), iters, float(tol), int(warm), _ptr(buf), _ptr(S))
+    if t < 0:
+        raise ValueError("oracle rejected the arguments")
+    return S, buf, int(t)
+
+
+def solve_ext(W, N, M, tau, iters, sweeps, tol=0.0, potentials=None, want_plan=False, want_mask=True,
+              threads=0):
+    """Matrix-level warm start / adaptive stopping.
+
+    potentials: None (cold) or (n_blocks, 2M) starting potentials (nats).
+    Returns dict(mask, potentials (n_blocks, 2M) fp64, iters_used (n_blocks,), plan, stats).
+    """
+    W = _f32(W)
+    rows, cols = W.shape
+    nb = (rows // M) * (cols // M)
+    warm = potentials is not None
+    uv = (np.array(potentials, dtype=np.float64).reshape(nb, 2 * M).copy() if warm
+          else np.zeros((nb, 2 * M), dtype=np.float64))
+    used = np.zeros(nb, dtype=np.int32)
+    plan_out = np.empty((rows, cols), dtype=np.float64) if want_plan else None
+    m = np.zeros((rows, words_per_row(cols)), dtype=np.uint32) if want_mask else None
+    st = Stats()
+    _check(lib().oracle_solve_ext(_ptr(W), rows, cols, N, M, float(tau), iters, sweeps, float(tol), int(warm),
+                                  _ptr(uv), _ptr(used), _ptr(plan_out), _ptr(m), threads, C.byref(st)))
+    return {"mask": m, "potentials": uv, "iters_used": used, "plan": plan_out, "stats": st.as_dict()}
 
 
 def unpack(mask_words, cols):

@@ -118,6 +118,69 @@ static void block_plan(const float* a, int N, int M, double tau, int iters,
     for (int e = 0; e < E; ++e) S_out[e] = exp(x[e]);
 }
 
+/* Warm start and adaptive stopping of the Dykstra loop.  The review fixes T
+ * and gives no convergence test ("Assumptions & free parameters"); these two
+ * extensions rest on one identity.  The row and column steps add potentials
+ * to x (r_i = ln N - LSE_i, c_j = ln N - LSE_j), and the clip only moves an
+ * amount between x and the correction q, so after every clip
+ *     x + q = y0 + U_i + V_j,   x = min(x + q, 0),   q = max(x + q, 0),
+ * where U, V are the potentials accumulated so far and y0 = x0 - tau.  The
+ * 2M numbers (U, V) are therefore the whole state of a block.
+ *  - Cold start: U = V = 0, i.e. x = y0 (<= 0), q = 0.  That is the start x0
+ *    of block_plan shifted by -tau in every row; the first row step removes
+ *    any per-row shift, so every later iterate equals block_plan's.
+ *  - Warm start: the caller's (U, V), e.g. the final potentials of an earlier
+ *    call on a nearby W.
+ *  - Stopping: after iteration t, with delta_t = the largest |r_i| and |c_j|
+ *    of that iteration, stop when tol > 0 and delta_t <= tol (at most iters
+ *    iterations).  tol = 0 runs all iters.
+ * uv (2M doubles, U then V): read when warm, always overwritten with the
+ * final potentials.  Returns the number of iterations run. */
+static int block_plan_ext(const float* a, int N, int M, double tau, int iters, double tol, int warm,
+                          double* uv, double* x, double* q, double* S_out) {
+    const int E = M * M;
+    double* U = uv;
+    double* V = uv + M;
+    if (!warm)
+        for (int k = 0; k < 2 * M; ++k) uv[k] = 0.0;
+    double mb = 0.0;
+    for (int e = 0; e < E; ++e) if ((double)a[e] > mb) mb = (double)a[e];
+    for (int i = 0; i < M; ++i)
+        for (int j = 0; j < M; ++j) {
+            const int e = i * M + j;
+            const double x0 = mb > 0.0 ? tau * ((double)a[e] / mb) : 0.0;
+            const double y = (x0 - tau) + U[i] + V[j];
+            x[e] = y < 0.0 ? y : 0.0;
+            q[e] = y - x[e];
+        }
+    const double lnN = log((double)N);
+    int t = 0;
+    while (t < iters) {
+        double delta = 0.0;
+        for (int i = 0; i < M; ++i) {
+            const double r = lnN - row_lse(x, M, i);
+            for (int j = 0; j < M; ++j) x[i * M + j] += r;
+            U[i] += r;
+            if (fabs(r) > delta) delta = fabs(r);
+        }
+        for (int j = 0; j < M; ++j) {
+            const double c = lnN - col_lse(x, M, j);
+            for (int i = 0; i < M; ++i) x[i * M + j] += c;
+            V[j] += c;
+            if (fabs(c) > delta) delta = fabs(c);
+        }
+        for (int e = 0; e < E; ++e) {
+            double y = x[e] + q[e];
+            x[e] = y < 0.0 ? y : 0.0;
+            q[e] = y - x[e];
+        }
+        ++t;
+        if (tol > 0.0 && delta <= tol) break;
+    }
+    for (int e = 0; e < E; ++e) S_out[e] = exp(x[e]);
+    return t;
+}
+
 /* ------------------------------------------------------------------ */
 /* Rounding (What carries the argument; Fig. 2 caption; referee comment 3). */
 
@@ -401,6 +464,17 @@ int oracle_block_round(const float* key, const float* a, int N, int M, int sweep
     return rc;
 }
 
+/* One block of block_plan_ext; returns the iterations run (or -1). */
+int oracle_block_plan_ext(const float* a, int N, int M, double tau, int iters, double tol, int warm,
+                          double* uv, double* S_out) {
+    if (check_args(M, M, N, M) || !(tol >= 0.0)) return -1;
+    double* x = (double*)malloc(sizeof(double) * M * M);
+    double* q = (double*)malloc(sizeof(double) * M * M);
+    int t = block_plan_ext(a, N, M, tau, iters, tol, warm, uv, x, q, S_out);
+    free(x); free(q);
+    return t;
+}
+
 double oracle_block_opt(const float* a, int N, int M, uint8_t* f) {
     if (check_args(M, M, N, M)) return NAN;
     return block_opt(a, N, M, f);
@@ -512,6 +586,70 @@ int oracle_mask(const float* W, int64_t rows, int64_t cols, int N, int M, double
     }
     pack_bits(bits, rows, cols, mask);
     free(bits);
+    if (st) { st->repairs += rep; st->ls_swaps += sw; st->failures += fail; st->short_after_greedy += shortg; }
+    return 0;
+}
+
+/* Full pipeline with warm start and adaptive stopping (block_plan_ext).
+ * uv: nb * 2M doubles, block b at 2M*b (U then V); read when warm, always
+ * overwritten (NaN for a block with non-finite W).  used_out (optional): nb
+ * ints, the iterations each block ran (0 for a non-finite block).
+ * plan_out (optional): rows*cols doubles.  mask (optional): when NULL the
+ * rounding is skipped. */
+int oracle_solve_ext(const float* W, int64_t rows, int64_t cols, int N, int M, double tau, int iters,
+                     int sweeps, double tol, int warm, double* uv, int* used_out, double* plan_out,
+                     uint32_t* mask, int threads, oracle_stats* st) {
+    int rc = check_args(rows, cols, N, M);
+    if (rc) return rc;
+    if (!(tol >= 0.0) || !uv) return -1;
+    const int64_t nbr = rows / M, nbc = cols / M, nb = nbr * nbc;
+    int64_t rep = 0, sw = 0, fail = 0, shortg = 0;
+    uint8_t* bits = mask ? (uint8_t*)malloc((size_t)(rows * cols > 0 ? rows * cols : 1)) : NULL;
+    set_threads(threads);
+#pragma omp parallel reduction(+:rep, sw, fail, shortg)
+    {
+        const int E = M * M;
+        float* a = (float*)malloc(sizeof(float) * E);
+        float* k = (float*)malloc(sizeof(float) * E);
+        double* x = (double*)malloc(sizeof(double) * E);
+        double* q = (double*)malloc(sizeof(double) * E);
+        double* S = (double*)malloc(sizeof(double) * E);
+        uint8_t* s = (uint8_t*)malloc((size_t)E);
+        int* order = (int*)malloc(sizeof(int) * E);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t b = 0; b < nb; ++b) {
+            int64_t br = b / nbc, bc = b % nbc;
+            double* buv = uv + 2 * M * b;
+            get_block(W, cols, M, br, bc, a);
+            oracle_stats l = {0, 0, 0, 0};
+            int ok = block_finite(a, E);
+            int used = 0;
+            if (ok) {
+                used = block_plan_ext(a, N, M, tau, iters, tol, warm, buv, x, q, S);
+            } else {
+                for (int e = 0; e < 2 * M; ++e) buv[e] = NAN;
+                for (int e = 0; e < E; ++e) S[e] = NAN;
+            }
+            if (used_out) used_out[b] = used;
+            if (plan_out)
+                for (int i = 0; i < M; ++i)
+                    for (int j = 0; j < M; ++j)
+                        plan_out[(br * M + i) * cols + bc * M + j] = S[i * M + j];
+            if (bits) {
+                if (ok) {
+                    for (int e = 0; e < E; ++e) k[e] = (float)S[e];
+                    ok = block_round(k, a, N, M, sweeps, 3, s, order, &l) == 0;
+                }
+                if (!ok) { memset(s, 0, (size_t)E); fail++; }
+                put_bits(bits, cols, M, br, bc, s);
+            } else if (!ok) {
+                fail++;
+            }
+            rep += l.repairs; sw += l.ls_swaps; shortg += l.short_after_greedy;
+        }
+        free(a); free(k); free(x); free(q); free(S); free(s); free(order);
+    }
+    if (bits) { pack_bits(bits, rows, cols, mask); free(bits); }
     if (st) { st->repairs += rep; st->ls_swaps += sw; st->failures += fail; st->short_after_greedy += shortg; }
     return 0;
 }
