@@ -72,8 +72,9 @@ typedef enum {
  * repair, local search, bit packing).
  *   mask_out: rows x words_per_row uint32, written completely.
  *   sweeps:   local-search sweeps L; one sweep visits every anchor row once.
- * Uses a stream-ordered workspace of rows*cols floats (cudaMallocAsync /
- * cudaFreeAsync on `stream`) that holds the plan between its two kernels.
+ * M = 16, 32, 64: one fused kernel, no workspace.  M = 4, 8: a plan kernel
+ * and a rounding kernel with a stream-ordered workspace of rows*cols floats
+ * between them (cudaMallocAsync / cudaFreeAsync on `stream`).
  */
 tsenor_status tsenor_mask(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
                           int N, int M, float tau, int iters, int sweeps,
@@ -151,6 +152,54 @@ tsenor_status tsenor_mask_safeguard(const void* W, tsenor_dtype dtype, int64_t r
 tsenor_status tsenor_mask_padded(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
                                  int N, int M, float tau, int iters, int sweeps,
                                  uint32_t* mask_out, tsenor_stream_t stream);
+
+/*
+ * tsenor_mask with warm start and adaptive stopping of the Dykstra loop.
+ *
+ * The review fixes the iteration count T and gives no convergence test
+ * ("Assumptions & free parameters"); inside an outer pruning loop the same
+ * layer is solved again and again for a slowly changing W.  This entry point
+ * lets such calls resume from the previous solution and stop each block once
+ * it has converged.  It rests on one identity: the row and column steps add
+ * potentials r_i = ln N - LSE_j(x_ij) and c_j = ln N - LSE_i(x_ij) to x, and
+ * the clip only moves an amount between x and its correction term, so after
+ * every iteration
+ *     x_ij + logQ_ij = (x0_ij - tau) + U_i + V_j,  x = min(that, 0),
+ * with U, V the potentials accumulated so far.  The 2M numbers (U, V) of a
+ * block are its whole Dykstra state.
+ *   potentials: (rows/M)*(cols/M) blocks x 2M fp32 (device), block b (row-major
+ *               over the block grid) at offset 2M*b: U_0..U_{M-1}, then
+ *               V_0..V_{M-1}, natural-log units.  warm != 0: read as the
+ *               starting state.  warm == 0: the start is U = V = 0 and the
+ *               array is only written (may be NULL then).  When non-NULL it is
+ *               overwritten with the final potentials (NaN for a block with
+ *               non-finite W).  The same array may be passed back on the next
+ *               call.
+ *   tol:        >= 0 and finite.  tol > 0: a block stops after the first
+ *               iteration whose potentials all satisfy |r_i| <= tol and
+ *               |c_j| <= tol (natural-log units; at most `iters`
+ *               iterations).  tol == 0: every block runs exactly `iters`.
+ *   iters_used: optional (rows/M)*(cols/M) int32 (device, may be NULL): the
+ *               iterations each block ran (0 for a non-finite block).
+ * With warm == 0 and tol == 0 the mask equals tsenor_mask's bit for bit.
+ * The stop decision is taken in fp32 on log2-scaled potentials, so a block
+ * whose largest step lies within about 1e-6 of tol may stop one iteration
+ * earlier or later than an exact evaluation would.
+ * Workspace as tsenor_mask.  The review has no counterpart of this call.
+ */
+tsenor_status tsenor_mask_warm(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
+                               int N, int M, float tau, int iters, int sweeps, float tol, int warm,
+                               float* potentials, int32_t* iters_used, uint32_t* mask_out,
+                               tsenor_stream_t stream);
+
+/*
+ * The plan of tsenor_mask_warm (same state, stop rule and outputs), written
+ * as tsenor_plan writes it.  Test hook and building block.
+ */
+tsenor_status tsenor_plan_warm(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
+                               int N, int M, float tau, int iters, float tol, int warm,
+                               float* potentials, int32_t* iters_used, float* plan_out,
+                               tsenor_stream_t stream);
 
 /* Static description of a status code. */
 const char* tsenor_status_string(int status);

@@ -18,7 +18,7 @@ STATUS = {0: "TSENOR_OK", -1: "TSENOR_ERR_ARG", -2: "TSENOR_ERR_SHAPE", -3: "TSE
 NOALLOC_MAX_PARAMS = 16 * 1024 * 1024
 EXPORTS = ("tsenor_mask", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
            "tsenor_status_string", "tsenor_last_error", "tsenor_mask_noalloc", "tsenor_mask_safeguard",
-           "tsenor_mask_padded")
+           "tsenor_mask_padded", "tsenor_mask_warm", "tsenor_plan_warm")
 
 _lib = None
 
@@ -43,6 +43,8 @@ def lib() -> C.CDLL:
         L.tsenor_plan.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, p, p]
         L.tsenor_mask_padded.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p]
         L.tsenor_mask_safeguard.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p, p, p]
+        L.tsenor_mask_warm.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, f32, i32, p, p, p, p]
+        L.tsenor_plan_warm.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, f32, i32, p, p, p, p]
         L.tsenor_round.argtypes = [p, p, i32, i64, i64, i32, i32, i32, p, p]
         L.tsenor_objective.argtypes = [p, i32, i64, i64, p, i32, i32, p, p]
         L.tsenor_error_count.argtypes = [p, C.POINTER(C.c_int64)]
@@ -152,6 +154,64 @@ def tsenor_mask_padded(W, N: int, M: int, tau: float, iters: int, sweeps: int, o
     return out
 
 
+def _warm_buffers(W, M, potentials, iters_used):
+    import torch
+    rows, cols = W.shape
+    nb = (rows // M) * (cols // M) if M > 0 and rows % M == 0 and cols % M == 0 else 0
+    if potentials is None:
+        potentials = torch.empty((nb, 2 * M), dtype=torch.float32, device=W.device)
+    elif (potentials.dtype != torch.float32 or not potentials.is_cuda or not potentials.is_contiguous()
+          or potentials.numel() < nb * 2 * M):
+        raise ValueError("potentials must be a contiguous float32 CUDA tensor of (n_blocks, 2M)")
+    if iters_used is None:
+        iters_used = torch.empty((nb,), dtype=torch.int32, device=W.device)
+    elif (iters_used.dtype != torch.int32 or not iters_used.is_cuda or not iters_used.is_contiguous()
+          or iters_used.numel() < nb):
+        raise ValueError("iters_used must be a contiguous int32 CUDA tensor of n_blocks")
+    return potentials, iters_used
+
+
+def tsenor_mask_warm(W, N: int, M: int, tau: float, iters: int, sweeps: int, tol: float = 0.0, potentials=None,
+                     warm: bool = False, iters_used=None, out=None, stream=None):
+    """tsenor_mask with warm start and adaptive stopping.
+
+    potentials: (n_blocks, 2M) float32 CUDA tensor, U then V per block
+    (natural-log units), read when ``warm`` and overwritten with the final
+    state (allocated when None; then ``warm`` must be False).  ``tol`` > 0
+    stops a block after the first iteration whose row and column potentials
+    are all within tol.  Returns (mask, potentials, iters_used).
+    """
+    import torch
+    _check_2d_cuda(W, "W")
+    rows, cols = W.shape
+    if warm and potentials is None:
+        raise ValueError("warm start needs potentials")
+    potentials, iters_used = _warm_buffers(W, M, potentials, iters_used)
+    if out is None:
+        out = torch.empty((rows, words_per_row(cols)), dtype=torch.int32, device=W.device)
+    _check(lib().tsenor_mask_warm(W.data_ptr(), _dtype_code(W), rows, cols, N, M, float(tau), iters, sweeps,
+                                  float(tol), int(bool(warm)), potentials.data_ptr(), iters_used.data_ptr(),
+                                  out.data_ptr(), _stream_handle(stream)))
+    return out, potentials, iters_used
+
+
+def tsenor_plan_warm(W, N: int, M: int, tau: float, iters: int, tol: float = 0.0, potentials=None,
+                     warm: bool = False, iters_used=None, out=None, stream=None):
+    """The plan of tsenor_mask_warm; returns (plan, potentials, iters_used)."""
+    import torch
+    _check_2d_cuda(W, "W")
+    rows, cols = W.shape
+    if warm and potentials is None:
+        raise ValueError("warm start needs potentials")
+    potentials, iters_used = _warm_buffers(W, M, potentials, iters_used)
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.float32, device=W.device)
+    _check(lib().tsenor_plan_warm(W.data_ptr(), _dtype_code(W), rows, cols, N, M, float(tau), iters, float(tol),
+                                  int(bool(warm)), potentials.data_ptr(), iters_used.data_ptr(), out.data_ptr(),
+                                  _stream_handle(stream)))
+    return out, potentials, iters_used
+
+
 def tsenor_plan(W, N: int, M: int, tau: float, iters: int, out=None, stream=None):
     """Fractional plan S (fp32, same shape as W) after `iters` Dykstra iterations."""
     import torch
@@ -198,5 +258,6 @@ def tsenor_error_count(stream=None) -> int:
     return int(n.value)
 
 
-__all__ = ["tsenor_mask", "tsenor_mask_noalloc", "tsenor_mask_safeguard", "tsenor_mask_padded", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
+__all__ = ["tsenor_mask", "tsenor_mask_noalloc", "tsenor_mask_safeguard", "tsenor_mask_padded", "tsenor_mask_warm",
+           "tsenor_plan", "tsenor_plan_warm", "tsenor_round", "tsenor_objective", "tsenor_error_count",
            "TsenorError", "lib", "words_per_row", "EXPORTS", "LIB_PATH"]

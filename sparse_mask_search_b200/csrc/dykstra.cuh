@@ -17,6 +17,14 @@
 //    one per column.
 //  * The plan is S = 2^min(y, 0) after the last iteration; S = 1 exactly
 //    for clipped entries (y >= 0).
+//  * Since y only ever gains r_i + c_j, y = y0 + U_i + V_j with U, V the
+//    potentials accumulated so far: the 2M numbers (U, V) are the whole
+//    state of a block.  The EXT kernels start from given (U, V) (warm
+//    start), export the final ones, and may stop a block early once every
+//    |r_i| and |c_j| of an iteration is at most a tolerance.  The review fixes
+//    T with no convergence test ("Assumptions & free parameters"); this is
+//    the library's extension, and U = V = 0 with no tolerance is exactly the
+//    plain solve.
 #pragma once
 
 #include "common.cuh"
@@ -24,6 +32,16 @@
 namespace tsenor {
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr double kLog2eD = 1.4426950408889634;
+constexpr double kLn2D = 0.6931471805599453;
+
+// Warm start / adaptive stopping arguments of the EXT kernels.
+struct DykstraExt {
+    float* potentials;      // [n_blocks][2M]: U_0..U_{M-1}, V_0..V_{M-1} (nats); in when warm, always out
+    int32_t* iters_used;    // [n_blocks] iterations run, or null
+    float tol2;             // stop tolerance on |r_i|, |c_j| in log2 units; 0 = run all iterations
+    int warm;               // nonzero: start from `potentials`
+};
 
 // Plan entry of one state value: S = 2^min(y, 0), exactly 1 when clipped.
 __device__ __forceinline__ float plan_value(float y) { return y >= 0.f ? 1.f : ex2(y); }
@@ -33,10 +51,10 @@ __device__ __forceinline__ float plan_value(float y) { return y >= 0.f ? 1.f : e
 // the exponentials of one row live only until its column contributions are
 // added, so no cross-thread traffic is needed at all.
 // ---------------------------------------------------------------------------
-template <int M, typename T>
+template <int M, typename T, bool EXT = false>
 __global__ void __launch_bounds__(128)
 dykstra_thread_kernel(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks,
-                      int N, float tau, int iters, float* __restrict__ plan) {
+                      int N, float tau, int iters, float* __restrict__ plan, DykstraExt ext = {}) {
     const int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
     if (b >= n_blocks) return;
     const int64_t nbc = cols / M;
@@ -73,8 +91,26 @@ dykstra_thread_kernel(const typename T::storage* __restrict__ W, int64_t cols, i
         }
     const float fN = float(N), log2N = log2f(float(N));
 
+    // EXT: accumulated potentials in log2 units, summed in fp64 so that the
+    // exported state carries no accumulation error of its own
+    double U[M], V[M];
+    int used = 0;
+    if constexpr (EXT) {
+        const float* uv = ext.warm ? ext.potentials + 2 * M * b : nullptr;
+#pragma unroll
+        for (int k = 0; k < M; ++k) {
+            U[k] = uv ? double(uv[k]) * kLog2eD : 0.0;
+            V[k] = uv ? double(uv[M + k]) * kLog2eD : 0.0;
+        }
+#pragma unroll
+        for (int i = 0; i < M; ++i)
+#pragma unroll
+            for (int j = 0; j < M; ++j) y[i][j] += float(U[i] + V[j]);
+    }
+
     if (finite) {
         for (int t = 0; t < iters; ++t) {
+            float delta = 0.f;                         // largest |r_i|, |c_j| of this iteration (EXT)
             float C[M];
 #pragma unroll
             for (int j = 0; j < M; ++j) C[j] = 0.f;
@@ -86,21 +122,38 @@ dykstra_thread_kernel(const typename T::storage* __restrict__ W, int64_t cols, i
                     e[j] = ex2(fminf(y[i][j], 0.f));
                     R += e[j];
                 }
-                const float w = fN * rcp(R);
+                const float w = fN * rcp_newton(R);
                 const float r = log2N - lg2(R);
 #pragma unroll
                 for (int j = 0; j < M; ++j) {
                     C[j] = fmaf(e[j], w, C[j]);
                     y[i][j] += r;
                 }
+                if constexpr (EXT) { U[i] += double(r); delta = fmaxf(delta, fabsf(r)); }
             }
 #pragma unroll
             for (int j = 0; j < M; ++j) {
                 const float c = log2N - lg2(C[j]);
 #pragma unroll
                 for (int i = 0; i < M; ++i) y[i][j] += c;
+                if constexpr (EXT) { V[j] += double(c); delta = fmaxf(delta, fabsf(c)); }
+            }
+            used = t + 1;
+            if constexpr (EXT) {
+                if (ext.tol2 > 0.f && delta <= ext.tol2) break;
             }
         }
+    }
+    if constexpr (EXT) {
+        if (ext.potentials) {
+            float* uv = ext.potentials + 2 * M * b;
+#pragma unroll
+            for (int k = 0; k < M; ++k) {
+                uv[k] = finite ? float(U[k] * kLn2D) : __int_as_float(0x7fc00000);
+                uv[M + k] = finite ? float(V[k] * kLn2D) : __int_as_float(0x7fc00000);
+            }
+        }
+        if (ext.iters_used) ext.iters_used[b] = finite ? used : 0;
     }
 #pragma unroll
     for (int i = 0; i < M; ++i) {
@@ -176,11 +229,14 @@ struct TileThread {
 // final state of this thread's sub-tile and `tile` the block's |W| (M x M in
 // shared memory, row stride TS).  Contains CTA-wide barriers: every thread of the CTA
 // must call it.  Returns whether the block's W is finite.
-template <int M, typename T, int TS = M>
+// EXT: warm start from / export to ext.potentials of block b, stop rule
+// ext.tol2, iteration count to ext.iters_used.
+template <int M, typename T, int TS = M, bool EXT = false>
 __device__ __forceinline__ bool dykstra_tile_solve(const typename T::storage* __restrict__ W, int64_t cols,
                                                    int64_t r0, int64_t c0, bool active, int N, float tau,
                                                    int iters, float* tile, float* colbuf,
-                                                   const TileThread<M>& th, float (&y)[4][8]) {
+                                                   const TileThread<M>& th, float (&y)[4][8],
+                                                   const DykstraExt& ext = DykstraExt{}, int64_t b = 0) {
     using C = TileCfg<M>;
     constexpr int P = C::P, Q = C::Q;
     const int lane = th.lane, warp = th.warp;
@@ -244,6 +300,31 @@ __device__ __forceinline__ bool dykstra_tile_solve(const typename T::storage* __
         }
     const float fN = float(N), log2N = log2f(float(N));
 
+    // EXT: y = y0 + U_i + V_j; this thread accumulates the potentials of the
+    // rows and columns it owns after the reduce-scatters (register k < RO
+    // holds row(k), register c < CO column col(c)).
+    // The sums are kept in fp64, so the exported state carries no
+    // accumulation error of its own.
+    double ua[C::RO], va[C::CO];
+    if constexpr (EXT) {
+        const float* uv = (ext.warm && active) ? ext.potentials + 2 * M * b : nullptr;
+        double U[P], V[Q];
+#pragma unroll
+        for (int k = 0; k < P; ++k) U[k] = uv ? double(uv[th.row(k)]) * kLog2eD : 0.0;
+#pragma unroll
+        for (int c = 0; c < Q; ++c) V[c] = uv ? double(uv[M + th.col(c)]) * kLog2eD : 0.0;
+#pragma unroll
+        for (int k = 0; k < P; ++k)
+#pragma unroll
+            for (int c = 0; c < Q; ++c) y[k][c] += float(U[k] + V[c]);
+#pragma unroll
+        for (int lo = 0; lo < C::RO; ++lo) ua[lo] = U[lo];
+#pragma unroll
+        for (int lo = 0; lo < C::CO; ++lo) va[lo] = V[lo];
+    }
+    bool done = !finite;                             // EXT: this block has stopped
+    int used = 0;
+
     // Blocks of one warp (M = 16) may differ in finiteness; all lanes run the
     // loop so that the shuffles stay converged, and a non-finite block's
     // result is discarded by the caller.
@@ -284,7 +365,7 @@ __device__ __forceinline__ bool dykstra_tile_solve(const typename T::storage* __
             float wv[P], rv[P];
 #pragma unroll
             for (int lo = 0; lo < C::RO; ++lo) {
-                wv[lo] = fN * rcp(rs[lo]);
+                wv[lo] = fN * (M <= 32 ? rcp_newton(rs[lo]) : rcp(rs[lo]));   // M = 64: the MUFU form timed faster
                 rv[lo] = log2N - lg2(rs[lo]);
             }
             // all-gather back into the permuted register order
@@ -338,11 +419,66 @@ __device__ __forceinline__ bool dykstra_tile_solve(const typename T::storage* __
                     for (int lo = 0; lo < C::CO; ++lo)
                         cv[(hi + s) * C::CO + lo] = __shfl_xor_sync(kFullMask, cv[hi * C::CO + lo], s * C::CG);
             // y += r_i + c_j
+            if constexpr (!EXT) {
 #pragma unroll
-            for (int k = 0; k < P; ++k)
+                for (int k = 0; k < P; ++k)
 #pragma unroll
-                for (int c = 0; c < Q2; ++c)
-                    y2[k][c] = add2(y2[k][c], add2(make_float2(rv[k], rv[k]), make_float2(cv[2 * c], cv[2 * c + 1])));
+                    for (int c = 0; c < Q2; ++c)
+                        y2[k][c] = add2(y2[k][c], add2(make_float2(rv[k], rv[k]), make_float2(cv[2 * c], cv[2 * c + 1])));
+            } else {
+                // a stopped block of a shared warp (M = 16) keeps its state
+                const float keep = done ? 0.f : 1.f;
+#pragma unroll
+                for (int k = 0; k < P; ++k)
+#pragma unroll
+                    for (int c = 0; c < Q2; ++c)
+                        y2[k][c] = fma2(make_float2(keep, keep),
+                                        add2(make_float2(rv[k], rv[k]), make_float2(cv[2 * c], cv[2 * c + 1])),
+                                        y2[k][c]);
+                float delta = 0.f;
+#pragma unroll
+                for (int lo = 0; lo < C::RO; ++lo) {
+                    if (!done) ua[lo] += double(rv[lo]);
+                    delta = fmaxf(delta, fabsf(rv[lo]));
+                }
+#pragma unroll
+                for (int lo = 0; lo < C::CO; ++lo) {
+                    if (!done) va[lo] += double(cv[lo]);
+                    delta = fmaxf(delta, fabsf(cv[lo]));
+                }
+                if (!done) used = it + 1;
+                if (ext.tol2 > 0.f) {
+                    const bool small = delta <= ext.tol2;
+                    bool all_small;
+                    if constexpr (C::TPB < 32) {
+                        const unsigned bal = __ballot_sync(kFullMask, small);
+                        const unsigned gm = ((1u << C::TPB) - 1u) << ((lane / C::TPB) * C::TPB);
+                        all_small = (bal & gm) == gm;
+                    } else if constexpr (C::TPB == 32) {
+                        all_small = __all_sync(kFullMask, small);
+                    } else {
+                        all_small = __syncthreads_and(small);
+                    }
+                    done = done || all_small;
+                    const bool stop = (C::TPB <= 32) ? (__all_sync(kFullMask, done) != 0) : done;
+                    if (stop) break;
+                }
+            }
+        }
+    }
+    if constexpr (EXT) {
+        if (active) {
+            if (ext.potentials) {
+                float* uv = ext.potentials + 2 * M * b;
+                const float nan = __int_as_float(0x7fc00000);
+                if (th.cg < C::RSR)
+#pragma unroll
+                    for (int lo = 0; lo < C::RO; ++lo) uv[th.row(lo)] = finite ? float(ua[lo] * kLn2D) : nan;
+                if (th.rg < C::RSC)
+#pragma unroll
+                    for (int lo = 0; lo < C::CO; ++lo) uv[M + th.col(lo)] = finite ? float(va[lo] * kLn2D) : nan;
+            }
+            if (ext.iters_used && th.t == 0) ext.iters_used[b] = finite ? used : 0;
         }
     }
 #pragma unroll
@@ -355,10 +491,10 @@ __device__ __forceinline__ bool dykstra_tile_solve(const typename T::storage* __
     return finite;
 }
 
-template <int M, typename T>
+template <int M, typename T, bool EXT = false>
 __global__ void __launch_bounds__(128)
 dykstra_tile_kernel(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks,
-                    int N, float tau, int iters, float* __restrict__ plan) {
+                    int N, float tau, int iters, float* __restrict__ plan, DykstraExt ext = {}) {
     using C = TileCfg<M>;
     extern __shared__ float smem[];
     const TileThread<M> th;
@@ -370,7 +506,8 @@ dykstra_tile_kernel(const typename T::storage* __restrict__ W, int64_t cols, int
     const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
 
     float y[C::P][C::Q];
-    const bool finite = dykstra_tile_solve<M, T>(W, cols, r0, c0, active, N, tau, iters, tile, colbuf, th, y);
+    const bool finite = dykstra_tile_solve<M, T, M, EXT>(W, cols, r0, c0, active, N, tau, iters, tile, colbuf, th, y,
+                                                         ext, b);
 
     // ---- plan via the smem tile, then 16-byte coalesced stores
     __syncthreads();

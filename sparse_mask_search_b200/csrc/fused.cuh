@@ -7,6 +7,8 @@
 //    to shared memory and rounds them one after another.
 //  - M = 64: one CTA of 4 warps per block; the CTA sorts, warp 0 runs the
 //    greedy and the repair, all 128 threads the local search.
+// EXT instances add the warm start, the stop rule and the potentials export
+// of dykstra_tile_solve.
 #pragma once
 
 #include <type_traits>
@@ -18,10 +20,10 @@ namespace tsenor {
 
 // bf16: registers capped for 5 CTAs (20 warps) per SM (5.00 ms against 5.03 ms
 // uncapped on the 4096x11008 16:32 workload); the fp32 key needs more.
-template <typename T>
+template <typename T, bool EXT = false>
 __global__ void __launch_bounds__(128, std::is_same<T, BF16>::value ? 5 : 4)
 fused_kernel32(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
-               int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr) {
+               int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr, DykstraExt ext = {}) {
     constexpr int M = 32;
     using C = TileCfg<M>;
     using Key = typename KeyOf<T>::type;
@@ -37,7 +39,8 @@ fused_kernel32(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
     const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
 
     float y[C::P][C::Q];
-    const bool finite = dykstra_tile_solve<M, T, TS>(W, cols, r0, c0, active, N, tau, iters, tile, nullptr, th, y);
+    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(W, cols, r0, c0, active, N, tau, iters, tile, nullptr, th,
+                                                          y, ext, b);
     if (!active) return;                              // no CTA-wide barrier follows
 
     Key key[C::P * C::Q];
@@ -60,10 +63,10 @@ constexpr size_t fused32_smem() {
 }
 
 // M = 16: a warp holds 4 blocks of 8 threads each.
-template <typename T>
+template <typename T, bool EXT = false>
 __global__ void __launch_bounds__(128)
 fused_kernel16(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
-               int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr) {
+               int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr, DykstraExt ext = {}) {
     constexpr int M = 16, TS = M + 1, E = M * M;
     using C = TileCfg<M>;
     using Key = typename KeyOf<T>::type;
@@ -82,7 +85,8 @@ fused_kernel16(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
     const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
 
     float y[C::P][C::Q];
-    const bool finite = dykstra_tile_solve<M, T, TS>(W, cols, r0, c0, active, N, tau, iters, tile, nullptr, th, y);
+    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(W, cols, r0, c0, active, N, tau, iters, tile, nullptr, th,
+                                                          y, ext, b);
     float* ptile = ptiles + th.blk * E;
 #pragma unroll
     for (int k = 0; k < C::P; ++k)
@@ -127,10 +131,10 @@ struct Fused64Smem {
     int ok;
 };
 
-template <typename T>
+template <typename T, bool EXT = false>
 __global__ void __launch_bounds__(128)
 fused_kernel64(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
-               int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr) {
+               int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr, DykstraExt ext = {}) {
     constexpr int M = 64, TS = M + 1;
     using C = TileCfg<M>;
     using Key = typename KeyOf<T>::type;
@@ -144,7 +148,8 @@ fused_kernel64(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
     const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
 
     float y[C::P][C::Q];
-    const bool finite = dykstra_tile_solve<M, T, TS>(W, cols, r0, c0, true, N, tau, iters, sm.a, sm.colbuf, th, y);
+    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(W, cols, r0, c0, true, N, tau, iters, sm.a, sm.colbuf, th,
+                                                          y, ext, b);
     Key key[C::P * C::Q];
 #pragma unroll
     for (int k = 0; k < C::P; ++k)

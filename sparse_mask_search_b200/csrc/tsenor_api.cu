@@ -35,22 +35,23 @@ tsenor_status check_common(const void* W, int dtype, int64_t rows, int64_t cols,
     return TSENOR_OK;
 }
 
-template <int M, typename T>
+// EXT = warm start / stop rule / potentials export (tsenor_mask_warm, tsenor_plan_warm).
+template <int M, typename T, bool EXT>
 cudaError_t launch_plan(const void* W, int64_t rows, int64_t cols, int N, float tau, int iters,
-                        float* plan, cudaStream_t st) {
+                        float* plan, cudaStream_t st, const DykstraExt& ext) {
     const int64_t nb = (rows / M) * (cols / M);
     const auto* w = static_cast<const typename T::storage*>(W);
     if constexpr (M <= 8) {
         const int64_t grid = (nb + 127) / 128;
-        dykstra_thread_kernel<M, T><<<dim3(unsigned(grid)), 128, 0, st>>>(w, cols, nb, N, tau, iters, plan);
+        dykstra_thread_kernel<M, T, EXT><<<dim3(unsigned(grid)), 128, 0, st>>>(w, cols, nb, N, tau, iters, plan, ext);
     } else {
         constexpr size_t smem = dykstra_tile_smem<M>();
-        cudaError_t e = cudaFuncSetAttribute(dykstra_tile_kernel<M, T>,
+        cudaError_t e = cudaFuncSetAttribute(dykstra_tile_kernel<M, T, EXT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
         const int64_t grid = (nb + TileCfg<M>::BPC - 1) / TileCfg<M>::BPC;
-        dykstra_tile_kernel<M, T><<<dim3(unsigned(grid)), TileCfg<M>::THREADS, smem, st>>>(
-            w, cols, nb, N, tau, iters, plan);
+        dykstra_tile_kernel<M, T, EXT><<<dim3(unsigned(grid)), TileCfg<M>::THREADS, smem, st>>>(
+            w, cols, nb, N, tau, iters, plan, ext);
     }
     return cudaGetLastError();
 }
@@ -85,58 +86,74 @@ cudaError_t launch_round(const float* plan, const void* W, int64_t rows, int64_t
 }
 
 // Whole path in one kernel (M = 16, 32, 64): no workspace.
-template <int M, typename T>
+template <int M, typename T, bool EXT>
 cudaError_t launch_fused(const void* W, int64_t rows, int64_t cols, int N, float tau, int iters, int sweeps,
-                         uint32_t* mask, cudaStream_t st) {
+                         uint32_t* mask, cudaStream_t st, const DykstraExt& ext) {
     const int64_t nb = (rows / M) * (cols / M);
     const int64_t wpr = (cols + 31) / 32;
     const auto* w = static_cast<const typename T::storage*>(W);
     cudaError_t e = cudaSuccess;
     if constexpr (M == 32) {
         constexpr size_t smem = fused32_smem();
-        e = cudaFuncSetAttribute(fused_kernel32<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        e = cudaFuncSetAttribute(fused_kernel32<T, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
-        fused_kernel32<T><<<dim3(unsigned((nb + 3) / 4)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps, mask,
-                                                                          wpr);
+        fused_kernel32<T, EXT><<<dim3(unsigned((nb + 3) / 4)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps,
+                                                                               mask, wpr, ext);
     } else if constexpr (M == 16) {
         if (cols % 32) {
             e = cudaMemsetAsync(mask, 0, size_t(rows) * size_t(wpr) * 4, st);   // padding bits
             if (e != cudaSuccess) return e;
         }
         constexpr size_t smem = fused16_smem();
-        e = cudaFuncSetAttribute(fused_kernel16<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        e = cudaFuncSetAttribute(fused_kernel16<T, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
-        fused_kernel16<T><<<dim3(unsigned((nb + 15) / 16)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps,
-                                                                            mask, wpr);
+        fused_kernel16<T, EXT><<<dim3(unsigned((nb + 15) / 16)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps,
+                                                                                 mask, wpr, ext);
     } else {
         constexpr size_t smem = sizeof(Fused64Smem<T>);
-        e = cudaFuncSetAttribute(fused_kernel64<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        e = cudaFuncSetAttribute(fused_kernel64<T, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
-        fused_kernel64<T><<<dim3(unsigned(nb)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps, mask, wpr);
+        fused_kernel64<T, EXT><<<dim3(unsigned(nb)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps, mask, wpr,
+                                                                     ext);
     }
     return cudaGetLastError();
 }
 
+// ext == nullptr: the plain solve; otherwise the EXT kernels with *ext.
+template <typename T, bool EXT>
+cudaError_t dispatch_fused_m(int M, const void* W, int64_t rows, int64_t cols, int N, float tau, int iters,
+                             int sweeps, uint32_t* mask, cudaStream_t st, const DykstraExt& ext) {
+    switch (M) {
+        case 16: return launch_fused<16, T, EXT>(W, rows, cols, N, tau, iters, sweeps, mask, st, ext);
+        case 32: return launch_fused<32, T, EXT>(W, rows, cols, N, tau, iters, sweeps, mask, st, ext);
+        default: return launch_fused<64, T, EXT>(W, rows, cols, N, tau, iters, sweeps, mask, st, ext);
+    }
+}
+
 template <typename T>
 cudaError_t dispatch_fused(int M, const void* W, int64_t rows, int64_t cols, int N, float tau, int iters, int sweeps,
-                           uint32_t* mask, cudaStream_t st) {
+                           uint32_t* mask, cudaStream_t st, const DykstraExt* ext = nullptr) {
+    return ext ? dispatch_fused_m<T, true>(M, W, rows, cols, N, tau, iters, sweeps, mask, st, *ext)
+               : dispatch_fused_m<T, false>(M, W, rows, cols, N, tau, iters, sweeps, mask, st, DykstraExt{});
+}
+
+template <typename T, bool EXT>
+cudaError_t dispatch_plan_m(int M, const void* W, int64_t rows, int64_t cols, int N, float tau, int iters,
+                            float* plan, cudaStream_t st, const DykstraExt& ext) {
     switch (M) {
-        case 16: return launch_fused<16, T>(W, rows, cols, N, tau, iters, sweeps, mask, st);
-        case 32: return launch_fused<32, T>(W, rows, cols, N, tau, iters, sweeps, mask, st);
-        default: return launch_fused<64, T>(W, rows, cols, N, tau, iters, sweeps, mask, st);
+        case 4: return launch_plan<4, T, EXT>(W, rows, cols, N, tau, iters, plan, st, ext);
+        case 8: return launch_plan<8, T, EXT>(W, rows, cols, N, tau, iters, plan, st, ext);
+        case 16: return launch_plan<16, T, EXT>(W, rows, cols, N, tau, iters, plan, st, ext);
+        case 32: return launch_plan<32, T, EXT>(W, rows, cols, N, tau, iters, plan, st, ext);
+        default: return launch_plan<64, T, EXT>(W, rows, cols, N, tau, iters, plan, st, ext);
     }
 }
 
 template <typename T>
 cudaError_t dispatch_plan(int M, const void* W, int64_t rows, int64_t cols, int N, float tau, int iters,
-                          float* plan, cudaStream_t st) {
-    switch (M) {
-        case 4: return launch_plan<4, T>(W, rows, cols, N, tau, iters, plan, st);
-        case 8: return launch_plan<8, T>(W, rows, cols, N, tau, iters, plan, st);
-        case 16: return launch_plan<16, T>(W, rows, cols, N, tau, iters, plan, st);
-        case 32: return launch_plan<32, T>(W, rows, cols, N, tau, iters, plan, st);
-        default: return launch_plan<64, T>(W, rows, cols, N, tau, iters, plan, st);
-    }
+                          float* plan, cudaStream_t st, const DykstraExt* ext = nullptr) {
+    return ext ? dispatch_plan_m<T, true>(M, W, rows, cols, N, tau, iters, plan, st, *ext)
+               : dispatch_plan_m<T, false>(M, W, rows, cols, N, tau, iters, plan, st, DykstraExt{});
 }
 
 template <typename T>
@@ -152,9 +169,9 @@ cudaError_t dispatch_round(int M, const float* plan, const void* W, int64_t rows
 }
 
 cudaError_t run_plan(int dtype, int M, const void* W, int64_t rows, int64_t cols, int N, float tau,
-                     int iters, float* plan, cudaStream_t st) {
-    return dtype == TSENOR_BF16 ? dispatch_plan<BF16>(M, W, rows, cols, N, tau, iters, plan, st)
-                                : dispatch_plan<F32>(M, W, rows, cols, N, tau, iters, plan, st);
+                     int iters, float* plan, cudaStream_t st, const DykstraExt* ext = nullptr) {
+    return dtype == TSENOR_BF16 ? dispatch_plan<BF16>(M, W, rows, cols, N, tau, iters, plan, st, ext)
+                                : dispatch_plan<F32>(M, W, rows, cols, N, tau, iters, plan, st, ext);
 }
 
 cudaError_t run_round(int dtype, int M, const float* plan, const void* W, int64_t rows, int64_t cols,
@@ -165,6 +182,15 @@ cudaError_t run_round(int dtype, int M, const float* plan, const void* W, int64_
 
 bool solver_params_ok(float tau, int iters) {
     return tau > 0.f && tau <= 3.0e38f && iters >= 1;
+}
+
+// Arguments of the warm-start entry points beyond the plain ones.
+bool warm_params_ok(float tol, int warm, const float* potentials, const int32_t* iters_used) {
+    if (!(tol >= 0.f) || tol > 3.0e38f) return false;            // NaN, negative or infinite
+    if (warm && !potentials) return false;
+    if (potentials && !aligned(potentials, 4)) return false;
+    if (iters_used && !aligned(iters_used, 4)) return false;
+    return true;
 }
 
 }  // namespace
@@ -218,6 +244,49 @@ extern "C" tsenor_status tsenor_mask(const void* W, tsenor_dtype dtype, int64_t 
     if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask launch");
     if (e2 != cudaSuccess) return cuda_fail(e2, "tsenor_mask workspace free");
     return TSENOR_OK;
+}
+
+extern "C" tsenor_status tsenor_mask_warm(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols, int N,
+                                          int M, float tau, int iters, int sweeps, float tol, int warm,
+                                          float* potentials, int32_t* iters_used, uint32_t* mask_out,
+                                          tsenor_stream_t stream) {
+    tsenor_status s = check_common(W, dtype, rows, cols, N, M);
+    if (s != TSENOR_OK) return s;
+    if (!solver_params_ok(tau, iters) || sweeps < 0) return TSENOR_ERR_ARG;
+    if (!warm_params_ok(tol, warm, potentials, iters_used)) return TSENOR_ERR_ARG;
+    if (rows == 0 || cols == 0) return TSENOR_OK;
+    if (!mask_out || !aligned(mask_out, 8)) return TSENOR_ERR_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const DykstraExt ext{potentials, iters_used, tol * kLog2e, warm != 0};
+    if (M >= 16) {
+        cudaError_t e = dtype == TSENOR_BF16
+                            ? dispatch_fused<BF16>(M, W, rows, cols, N, tau, iters, sweeps, mask_out, st, &ext)
+                            : dispatch_fused<F32>(M, W, rows, cols, N, tau, iters, sweeps, mask_out, st, &ext);
+        return e == cudaSuccess ? TSENOR_OK : cuda_fail(e, "tsenor_mask_warm launch");
+    }
+    float* plan = nullptr;
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&plan), size_t(rows) * size_t(cols) * sizeof(float), st);
+    if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask_warm workspace");
+    e = run_plan(dtype, M, W, rows, cols, N, tau, iters, plan, st, &ext);
+    if (e == cudaSuccess) e = run_round(dtype, M, plan, W, rows, cols, N, sweeps, mask_out, st);
+    cudaError_t e2 = cudaFreeAsync(plan, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask_warm launch");
+    if (e2 != cudaSuccess) return cuda_fail(e2, "tsenor_mask_warm workspace free");
+    return TSENOR_OK;
+}
+
+extern "C" tsenor_status tsenor_plan_warm(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols, int N,
+                                          int M, float tau, int iters, float tol, int warm, float* potentials,
+                                          int32_t* iters_used, float* plan_out, tsenor_stream_t stream) {
+    tsenor_status s = check_common(W, dtype, rows, cols, N, M);
+    if (s != TSENOR_OK) return s;
+    if (!solver_params_ok(tau, iters)) return TSENOR_ERR_ARG;
+    if (!warm_params_ok(tol, warm, potentials, iters_used)) return TSENOR_ERR_ARG;
+    if (rows == 0 || cols == 0) return TSENOR_OK;
+    if (!plan_out || !aligned(plan_out, 16)) return TSENOR_ERR_ARG;
+    const DykstraExt ext{potentials, iters_used, tol * kLog2e, warm != 0};
+    cudaError_t e = run_plan(dtype, M, W, rows, cols, N, tau, iters, plan_out, (cudaStream_t)stream, &ext);
+    return e == cudaSuccess ? TSENOR_OK : cuda_fail(e, "tsenor_plan_warm launch");
 }
 
 extern "C" tsenor_status tsenor_mask_safeguard(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,

@@ -73,6 +73,34 @@ def test_other_entry_points_validate():
     assert L.tsenor_error_count(None, None) == -1
 
 
+def _warm(L, W=1 << 12, rows=64, cols=64, N=2, M=4, tau=10.0, iters=5, sweeps=1, tol=0.0, warm=0, pot=1 << 12,
+          used=1 << 12, out=1 << 12):
+    return L.tsenor_mask_warm(W, 1, rows, cols, N, M, tau, iters, sweeps, tol, warm, pot, used, out, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(tol=-1e-3), -1), (dict(tol=float("nan")), -1), (dict(tol=float("inf")), -1),
+    (dict(warm=1, pot=0), -1), (dict(pot=(1 << 12) + 2), -1), (dict(used=(1 << 12) + 1), -1),
+    (dict(out=0), -1), (dict(iters=0), -1), (dict(M=12), -3), (dict(cols=66), -2),
+])
+def test_warm_entry_points_validate(kw, code):
+    L = tsl.lib()
+    assert _warm(L, **kw) == code
+    plan_kw = {k: v for k, v in kw.items() if k not in ("sweeps", "out")}
+    if "out" not in kw:
+        a = dict(W=1 << 12, rows=64, cols=64, N=2, M=4, tau=10.0, iters=5, tol=0.0, warm=0, pot=1 << 12,
+                 used=1 << 12, out=1 << 12)
+        a.update(plan_kw)
+        assert L.tsenor_plan_warm(a["W"], 1, a["rows"], a["cols"], a["N"], a["M"], a["tau"], a["iters"], a["tol"],
+                                  a["warm"], a["pot"], a["used"], a["out"], None) == code
+
+
+def test_warm_empty_calls_do_nothing():
+    L = tsl.lib()
+    assert _warm(L, rows=0, W=0, out=0, pot=0, used=0) == 0
+    assert L.tsenor_plan_warm(0, 1, 0, 64, 2, 4, 10.0, 5, 0.0, 0, None, None, None, None) == 0
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(tsl, "_lib", None)
     monkeypatch.setattr(tsl, "LIB_PATH", str(tmp_path / "missing.so"))

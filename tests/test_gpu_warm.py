@@ -1,0 +1,214 @@
+"""Warm start and adaptive stopping (tsenor_mask_warm / tsenor_plan_warm)
+against the oracle's block_plan_ext.
+
+The review fixes T and gives no convergence test ("Assumptions & free
+parameters"); the extension carries the Dykstra state as the accumulated row
+and column potentials (U, V) and stops a block at the first iteration whose
+largest potential step is <= tol.  Bars:
+  - cold start, tol = 0: the plain solve bit for bit (same kernels' arithmetic);
+  - plans within PLAN_TOL of the oracle's fp64 plans;
+  - the exported state U_i + V_j (what a restart uses) within STATE_TOL of
+    the oracle's: a restart then moves the plan by at most STATE_TOL
+    (d exp(y)/dy <= 1 for y <= 0), well inside PLAN_TOL;
+  - each potential on its own within gauge_tol(M, T): (U + k, V - k) is the
+    same state, and nothing in the iteration pulls that direction back, so
+    the fp32 rounding of the M-term row and column sums (about M 2^-24 per
+    iteration, random sign) walks U and V apart by about sqrt(T) M 2^-24;
+    the kernels sum the potentials themselves in fp64;
+  - masks identical to the oracle's wherever the stop iteration agrees;
+  - the stop iteration agrees with the oracle's except where the oracle's
+    step at the deciding iteration lies within STOP_SLACK of tol: the kernel
+    takes that decision in fp32 on log2-scaled potentials.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import PLAN_TOL, block_bits, mask_to_np, record, to_device
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import sparse_mask_search_b200 as tsl  # noqa: E402
+
+STATE_TOL = 5e-5         # max |(U_i + V_j)_gpu - (U_i + V_j)_oracle| (nats)
+STOP_SLACK = 2e-6        # fp32 error of a potential step, nats
+
+
+def gauge_tol(M, T):
+    return 4.0 * np.sqrt(T) * M * 2.0 ** -24 * np.log(2.0) + 1e-5
+
+
+def pot_errors(pot_gpu, pot_ref, M, rows=None):
+    """(max error of the state U_i + V_j, max error of a single potential) over the given blocks."""
+    g = np.asarray(pot_gpu, dtype=np.float64).reshape(-1, 2 * M)
+    r = np.asarray(pot_ref, dtype=np.float64).reshape(-1, 2 * M)
+    if rows is not None:
+        g, r = g[rows], r[rows]
+    d = g - r
+    state = np.abs(d[:, :M, None] + d[:, None, M:])
+    return float(state.max()), float(np.abs(d).max())
+
+CASES = [  # M, N, dtype, dist, rows, cols, tau, iters, sweeps
+    (4, 2, "f32", "normal", 16, 40, 10.0, 200, 1),
+    (8, 4, "bf16", "t3_outlier_cols", 32, 48, 20.0, 200, 4),
+    (16, 8, "bf16", "t3_outlier_cols", 48, 80, 20.0, 300, 4),
+    (16, 5, "f32", "normal", 32, 64, 20.0, 300, 4),
+    (32, 16, "bf16", "t3_outlier_cols", 64, 96, 20.0, 300, 8),
+    (32, 16, "f32", "normal", 32, 64, 20.0, 300, 8),
+    (64, 32, "bf16", "laplace_outliers", 128, 192, 30.0, 400, 8),
+]
+IDS = [f"{c[2]}-{c[1]}of{c[0]}" for c in CASES]
+
+
+def _setup(case, seed=0):
+    M, N, dtype, dist, rows, cols, tau, iters, sweeps = case
+    stor, W = synth.make_matrix(rows, cols, dtype, dist, 0.02, seed=seed + M + rows)
+    return M, N, dtype, rows, cols, tau, iters, sweeps, stor, W
+
+
+def _plan_blocks(P, M):
+    return oracle.blocks_view(np.asarray(P, dtype=np.float64), M).reshape(-1, M, M)
+
+
+@pytest.mark.parametrize("case", CASES, ids=IDS)
+def test_cold_start_equals_plain_solve(case):
+    M, N, dtype, rows, cols, tau, iters, sweeps, stor, W = _setup(case)
+    Wd = to_device(stor, dtype)
+    ref_mask = tsl.tsenor_mask(Wd, N, M, tau, iters, sweeps)
+    ref_plan = tsl.tsenor_plan(Wd, N, M, tau, iters)
+    mask, pot, used = tsl.tsenor_mask_warm(Wd, N, M, tau, iters, sweeps)
+    plan, pot2, used2 = tsl.tsenor_plan_warm(Wd, N, M, tau, iters)
+    assert torch.equal(mask, ref_mask)
+    assert torch.equal(plan, ref_plan)
+    assert torch.equal(pot, pot2) and torch.equal(used, used2)
+    assert (used.cpu().numpy() == iters).all()
+    ores = oracle.solve_ext(W, N, M, tau, iters, sweeps, want_plan=True, want_mask=False)
+    dstate, dpot = pot_errors(pot.cpu().numpy(), ores["potentials"], M)
+    record(f"warm-cold-{IDS[CASES.index(case)]}", {"state_max_abs": dstate, "pot_max_abs": dpot,
+                                                   "gauge_tol": gauge_tol(M, iters)})
+    assert dstate <= STATE_TOL
+    assert dpot <= gauge_tol(M, iters)
+
+
+@pytest.mark.parametrize("case", CASES, ids=IDS)
+def test_warm_start_matches_oracle(case):
+    M, N, dtype, rows, cols, tau, iters, sweeps, stor, W = _setup(case, seed=1)
+    Wd = to_device(stor, dtype)
+    t1, t2 = iters // 3, iters - iters // 3
+    # starting state: the oracle's potentials after t1 iterations, rounded to fp32 for both sides
+    start = oracle.solve_ext(W, N, M, tau, t1, sweeps, want_mask=False)["potentials"].astype(np.float32)
+    ores = oracle.solve_ext(W, N, M, tau, t2, sweeps, potentials=start.astype(np.float64), want_plan=True)
+    pot = torch.from_numpy(start.copy()).cuda()
+    plan, pot_p, _ = tsl.tsenor_plan_warm(Wd, N, M, tau, t2, potentials=pot.clone(), warm=True)
+    mask, pot_m, used = tsl.tsenor_mask_warm(Wd, N, M, tau, t2, sweeps, potentials=pot, warm=True)
+    assert torch.equal(pot_p, pot_m)
+    assert (used.cpu().numpy() == t2).all()
+    dplan = float(np.abs(plan.cpu().numpy().astype(np.float64) - ores["plan"]).max())
+    dstate, dpot = pot_errors(pot_m.cpu().numpy(), ores["potentials"], M)
+    bg, br = block_bits(mask_to_np(mask), cols, M), block_bits(ores["mask"], cols, M)
+    same = float((bg == br).all(axis=(2, 3)).mean())
+    record(f"warm-start-{IDS[CASES.index(case)]}", {"plan_max_abs": dplan, "state_max_abs": dstate,
+                                                    "pot_max_abs": dpot, "same_blocks": same})
+    assert dplan <= PLAN_TOL
+    assert dstate <= STATE_TOL and dpot <= gauge_tol(M, t2)
+    assert (bg.sum(axis=3) == N).all() and (bg.sum(axis=2) == N).all()
+    assert same == 1.0
+    # the mask is the rounding of the exported plan
+    assert torch.equal(mask, tsl.tsenor_round(plan, Wd, N, M, sweeps))
+
+
+def _step(a, N, tau, k, start):
+    """Largest |r_i|, |c_j| of iteration k of the oracle (potentials after k minus after k-1)."""
+    _, uk, _ = oracle.block_plan_ext(a, N, tau, k, uv=start)
+    if k == 1:
+        base = start if start is not None else np.zeros(2 * a.shape[0])
+    else:
+        _, base, _ = oracle.block_plan_ext(a, N, tau, k - 1, uv=start)
+    return float(np.abs(uk - base).max())
+
+
+@pytest.mark.parametrize("tol", [1e-3, 1e-4])
+@pytest.mark.parametrize("case", CASES, ids=IDS)
+def test_adaptive_stop_matches_oracle(case, tol):
+    M, N, dtype, rows, cols, tau, iters, sweeps, stor, W = _setup(case, seed=2)
+    iters = 3000                                          # a cap the stop rule reaches first
+    W = W.copy()
+    stor = np.ascontiguousarray(stor).copy()
+    stor[:M, M:2 * M] = 0                                 # a zero block converges at once
+    W[:M, M:2 * M] = 0.0
+    Wd = to_device(stor, dtype)
+    plan, pot, used = tsl.tsenor_plan_warm(Wd, N, M, tau, iters, tol=tol)
+    mask, pot_m, used_m = tsl.tsenor_mask_warm(Wd, N, M, tau, iters, sweeps, tol=tol)
+    assert torch.equal(pot, pot_m) and torch.equal(used, used_m)
+    ores = oracle.solve_ext(W, N, M, tau, iters, sweeps, tol=tol, want_plan=True)
+    ug, uo = used.cpu().numpy(), ores["iters_used"]
+    assert (uo < iters).all()
+    blocks_a = oracle.blocks_view(np.abs(W), M).reshape(-1, M, M)
+    differ = np.nonzero(ug != uo)[0]
+    for b in differ:
+        # a different stop iteration only where the oracle's step at the deciding iteration is within slack of tol
+        k = int(min(ug[b], uo[b]))
+        assert abs(int(ug[b]) - int(uo[b])) == 1, (b, ug[b], uo[b])
+        assert abs(_step(blocks_a[b], N, tau, k, None) - tol) <= STOP_SLACK, b
+    agree = ug == uo
+    Pg, Po = _plan_blocks(plan.cpu().numpy(), M), _plan_blocks(ores["plan"], M)
+    dplan = float(np.abs(Pg[agree] - Po[agree]).max())
+    dstate, dpot = pot_errors(pot.cpu().numpy(), ores["potentials"], M, rows=agree)
+    bg = block_bits(mask_to_np(mask), cols, M).reshape(-1, M, M)
+    br = block_bits(ores["mask"], cols, M).reshape(-1, M, M)
+    record(f"warm-stop-{tol:g}-{IDS[CASES.index(case)]}",
+           {"plan_max_abs": dplan, "state_max_abs": dstate, "pot_max_abs": dpot,
+            "stop_mismatch": int(len(differ)), "blocks": int(len(ug)), "mean_iters": float(ug.mean())})
+    assert len(differ) <= max(1, len(ug) // 100)
+    assert dplan <= PLAN_TOL and dstate <= STATE_TOL and dpot <= gauge_tol(M, int(uo.max()))
+    assert (bg[agree] == br[agree]).all()
+    assert (bg.sum(axis=2) == N).all() and (bg.sum(axis=1) == N).all()
+
+
+@pytest.mark.parametrize("case", [CASES[1], CASES[2], CASES[4], CASES[6]], ids=[IDS[1], IDS[2], IDS[4], IDS[6]])
+def test_restart_continues_the_run(case):
+    """GPU against itself: T1 iterations, then T2 more from the exported
+    potentials, is the run of T1 + T2 (the potentials are the whole state)."""
+    M, N, dtype, rows, cols, tau, iters, sweeps, stor, W = _setup(case, seed=3)
+    Wd = to_device(stor, dtype)
+    t1 = iters // 2
+    plan_all, pot_all, _ = tsl.tsenor_plan_warm(Wd, N, M, tau, iters)
+    _, pot1, _ = tsl.tsenor_plan_warm(Wd, N, M, tau, t1)
+    plan2, pot2, _ = tsl.tsenor_plan_warm(Wd, N, M, tau, iters - t1, potentials=pot1, warm=True)
+    assert float((plan2 - plan_all).abs().max()) <= PLAN_TOL
+    dstate, dpot = pot_errors(pot2.cpu().numpy(), pot_all.cpu().numpy(), M)
+    assert dstate <= 2 * STATE_TOL and dpot <= 2 * gauge_tol(M, iters)
+
+
+def test_converged_warm_start_stops_after_one_iteration():
+    M, N, tau = 32, 16, 20.0
+    stor, W = synth.make_matrix(64, 128, "bf16", "t3_outlier_cols", 0.02, seed=11)
+    Wd = to_device(stor, "bf16")
+    mask, pot, used = tsl.tsenor_mask_warm(Wd, N, M, tau, 5000, 8, tol=1e-5)
+    assert (used.cpu().numpy() < 5000).all()
+    mask2, pot2, used2 = tsl.tsenor_mask_warm(Wd, N, M, tau, 5000, 8, tol=1e-3, potentials=pot.clone(), warm=True)
+    assert (used2.cpu().numpy() == 1).all()
+    same = (block_bits(mask_to_np(mask), 128, M) == block_bits(mask_to_np(mask2), 128, M)).all(axis=(2, 3))
+    assert same.mean() >= 0.9
+
+
+@pytest.mark.parametrize("M,N", [(8, 4), (16, 8), (32, 16), (64, 32)])
+def test_non_finite_block(M, N):
+    stor, W = synth.make_matrix(2 * M, 3 * M, "f32", "normal", 0.02, seed=M)
+    stor = np.ascontiguousarray(stor).copy()
+    stor[1, M + 2] = np.nan                                 # block (0, 1)
+    Wd = to_device(stor, "f32")
+    tsl.tsenor_error_count()                                # reset the failure counter
+    mask, pot, used = tsl.tsenor_mask_warm(Wd, N, M, 20.0, 100, 2, tol=1e-4)
+    assert tsl.tsenor_error_count() == 1
+    p, u = pot.cpu().numpy(), used.cpu().numpy()
+    assert np.isnan(p[1]).all() and u[1] == 0
+    assert np.isfinite(np.delete(p, 1, axis=0)).all() and (np.delete(u, 1) > 0).all()
+    bits = block_bits(mask_to_np(mask), 3 * M, M)
+    assert bits[0, 1].sum() == 0
+    ores = oracle.solve_ext(stor, N, M, 20.0, 100, 2, tol=1e-4)
+    ok = u == ores["iters_used"]
+    br = block_bits(ores["mask"], 3 * M, M).reshape(-1, M, M)
+    assert (bits.reshape(-1, M, M)[ok] == br[ok]).all()
