@@ -52,7 +52,7 @@ fused_kernel32(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
             key[k * C::Q + c] = Key::make(plan_value(y[k][c]), tile[th.row(k) * TS + th.col(c)], e);
         }
     bool ok = finite;                                 // one block per warp: uniform
-    if (ok) ok = round_block_warp<M, Key>(key, tile, shs[th.blk], N, sweeps, th.lane);
+    if (ok) ok = round_block_warp<M, Key>(key, tile, shs[th.blk].view(), N, sweeps, th.lane);
     if (!ok && th.lane == 0) atomicAdd(&g_block_failures, 1ull);
     __syncwarp();
     write_mask_rows<M>(mask, wpr, r0, c0, shs[th.blk].rowbits, ok, th.lane);
@@ -110,7 +110,7 @@ fused_kernel16(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
             key[r] = Key::make(pt[e], at[(e / M) * TS + (e % M)], e);
         }
         bool ok = flags[slot] != 0;
-        if (ok) ok = round_block_warp<M, Key>(key, at, shs[warp], N, sweeps, lane);
+        if (ok) ok = round_block_warp<M, Key>(key, at, shs[warp].view(), N, sweeps, lane);
         if (!ok && lane == 0) atomicAdd(&g_block_failures, 1ull);
         __syncwarp();
         write_mask_rows<M>(mask, wpr, rr, cc, shs[warp].rowbits, ok, lane);
@@ -122,14 +122,9 @@ constexpr size_t fused16_smem() {
     return sizeof(float) * 16 * (16 * 17 + 16 * 16) + sizeof(RoundShared<16>) * 4 + sizeof(int) * 16;
 }
 
-// M = 64: one CTA of 4 warps per block.
-template <typename T>
-struct Fused64Smem {
-    RoundCta64Work<typename KeyOf<T>::type> u;
-    float a[64 * 65];                                   // |W|, row stride 65
-    float colbuf[2 * 4 * 32 * TileCfg<64>::CO];         // cross-warp column sums
-    int ok;
-};
+// M = 64: one CTA of 4 warps per block; Round64Smem's colbuf serves the
+// Dykstra phase's cross-warp column sums.
+static_assert(Round64Smem<KeyB>::kColbufFloats >= 2 * 4 * 32 * TileCfg<64>::CO, "column-sum buffer");
 
 template <typename T, bool EXT = false>
 __global__ void __launch_bounds__(128)
@@ -140,7 +135,7 @@ fused_kernel64(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
     using Key = typename KeyOf<T>::type;
     static_assert(C::TPB == 128 && C::BPC == 1, "one block per CTA");
     extern __shared__ __align__(16) unsigned char fused64_raw[];
-    Fused64Smem<T>& sm = *reinterpret_cast<Fused64Smem<T>*>(fused64_raw);
+    Round64Smem<Key>& sm = *reinterpret_cast<Round64Smem<Key>*>(fused64_raw);
     const TileThread<M> th;
     const int64_t b = blockIdx.x;
     if (b >= n_blocks) return;                         // uniform per CTA
@@ -148,8 +143,8 @@ fused_kernel64(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
     const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
 
     float y[C::P][C::Q];
-    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(W, cols, r0, c0, true, N, tau, iters, sm.a, sm.colbuf, th,
-                                                          y, ext, b);
+    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(W, cols, r0, c0, true, N, tau, iters, sm.a, sm.v.colbuf,
+                                                          th, y, ext, b);
     Key key[C::P * C::Q];
 #pragma unroll
     for (int k = 0; k < C::P; ++k)
@@ -159,9 +154,9 @@ fused_kernel64(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
             key[k * C::Q + c] = Key::make(plan_value(y[k][c]), sm.a[row * TS + col], row * M + col);
         }
     bool ok = finite;                                   // uniform over the CTA
-    if (ok) ok = round_block_cta64(key, sm.a, sm.u, &sm.ok, N, sweeps, th.tid);
+    if (ok) ok = round_block_cta64(key, sm, N, sweeps, th.tid);
     if (!ok && th.tid == 0) atomicAdd(&g_block_failures, 1ull);
-    write_mask_rows<M>(mask, wpr, r0, c0, sm.u.sh.rowbits, ok, th.tid, 128);
+    write_mask_rows<M>(mask, wpr, r0, c0, sm.v.rb.rowbits, ok, th.tid, 128);
 }
 
 }  // namespace tsenor

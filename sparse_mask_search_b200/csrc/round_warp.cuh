@@ -88,18 +88,34 @@ __device__ __forceinline__ int lowest_bit(Bits x) {
     else return __ffs(static_cast<int>(x)) - 1;
 }
 
-// Per-block shared memory of the rounding steps after the sort.
+// Where the rounding steps after the sort keep one block's state (shared
+// memory).  A view of pointers, so that M = 64 can overlay the arrays of
+// different steps (see Round64Smem).
+template <int M>
+struct RoundView {
+    using Bits = typename WarpRound<M>::Bits;
+    float* G;                           // cached pair gains (local search), row stride M+1
+    uint16_t* order;                    // sorted flat indices
+    Bits* rowbits;                      // row bitmasks of the mask being built
+    float* bestv;                       // best gain of each row over its partners ...
+    int* bestp;                         // ... and that partner (lowest index on ties)
+    int* rc;                            // row counts (greedy, repair)
+    int* cc;                            // column counts
+};
+
+// Per-block shared memory of the rounding steps after the sort (M <= 32).
 template <int M>
 struct RoundShared {
     using Bits = typename WarpRound<M>::Bits;
     static constexpr int GS = M + 1;
-    float G[M * GS];                    // cached pair gains (local search), row stride M+1
-    uint16_t order[WarpRound<M>::EP];   // sorted flat indices
+    float G[M * GS];
+    uint16_t order[WarpRound<M>::EP];
     Bits rowbits[M];
-    float bestv[M];                     // best gain of each row over its partners ...
-    int bestp[M];                       // ... and that partner (lowest index on ties)
+    float bestv[M];
+    int bestp[M];
     int rc[M];
     int cc[M];
+    __device__ __forceinline__ RoundView<M> view() { return RoundView<M>{G, order, rowbits, bestv, bestp, rc, cc}; }
 };
 
 // Bitonic compare-exchange of registers r and r|J of this lane: the pair ends
@@ -224,7 +240,7 @@ __device__ __forceinline__ void warp_argmax(float& v, int& i) {
 
 // Sorted keys of one warp into sh.order.
 template <int M, typename Key>
-__device__ __forceinline__ void keys_to_order(const Key (&key)[WarpRound<M>::R], RoundShared<M>& sh, int lane) {
+__device__ __forceinline__ void keys_to_order(const Key (&key)[WarpRound<M>::R], const RoundView<M>& sh, int lane) {
     constexpr int R = WarpRound<M>::R, E = M * M;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -236,7 +252,7 @@ __device__ __forceinline__ void keys_to_order(const Key (&key)[WarpRound<M>::R],
 // Steps 2-3 (greedy, repair) for one block by one warp, from sh.order.
 // Returns false when the block could not be made feasible.
 template <int M, int EP>
-__device__ bool greedy_and_repair(const float* a, RoundShared<M>& sh, int N, int lane) {
+__device__ bool greedy_and_repair(const float* a, const RoundView<M>& sh, int N, int lane) {
     using Bits = typename WarpRound<M>::Bits;
     constexpr int E = M * M, AS = M + 1;
     for (int r = lane; r < M; r += 32) { sh.rc[r] = 0; sh.cc[r] = 0; sh.rowbits[r] = 0; }
@@ -358,7 +374,7 @@ __device__ __forceinline__ float row_max(float t) {
 
 // Best partner of row x over the cached gains (lowest partner index on ties).
 template <int M>
-__device__ __forceinline__ void rescan_row(RoundShared<M>& sh, int x) {
+__device__ __forceinline__ void rescan_row(const RoundView<M>& sh, int x) {
     constexpr int GS = M + 1;
     float g[M];
 #pragma unroll
@@ -377,7 +393,7 @@ __device__ __forceinline__ void rescan_row(RoundShared<M>& sh, int x) {
 // Step 4 for one block by LsCfg<M>::NT threads: the gain table, the row
 // bests, then the sweeps.  `a`: |W| with row stride M+1.
 template <int M>
-__device__ void local_search(const float* a, RoundShared<M>& sh, int sweeps, int tid) {
+__device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps, int tid) {
     using L = LsCfg<M>;
     using Bits = typename WarpRound<M>::Bits;
     constexpr int AS = M + 1, GS = M + 1, NT = L::NT, CH = L::CH, CPT = L::CPT;
@@ -482,7 +498,7 @@ __device__ void local_search(const float* a, RoundShared<M>& sh, int sweeps, int
 // Returns false when the block could not be made feasible (never expected,
 // see the repair proof); the final row bitmasks are in sh.rowbits.
 template <int M, typename Key>
-__device__ bool round_block_warp(Key (&key)[WarpRound<M>::R], const float* a, RoundShared<M>& sh, int N,
+__device__ bool round_block_warp(Key (&key)[WarpRound<M>::R], const float* a, const RoundView<M>& sh, int N,
                                  int sweeps, int lane) {
     constexpr int R = WarpRound<M>::R;
     warp_bitonic_sort<R>(key, lane);
@@ -564,7 +580,7 @@ round_warp_kernel(const float* __restrict__ plan, const typename T::storage* __r
     }
     ok = __all_sync(kFullMask, ok);
     __syncwarp();
-    if (ok) ok = round_block_warp<M, Key>(key, sm.a, sm.sh, N, sweeps, lane);
+    if (ok) ok = round_block_warp<M, Key>(key, sm.a, sm.sh.view(), N, sweeps, lane);
     if (!ok && lane == 0) atomicAdd(&g_block_failures, 1ull);
     __syncwarp();
     write_mask_rows<M>(mask, wpr, r0, c0, sm.sh.rowbits, ok, lane);
@@ -573,47 +589,251 @@ round_warp_kernel(const float* __restrict__ plan, const typename T::storage* __r
 template <int M>
 constexpr size_t round_warp_smem() { return sizeof(RoundWarpSmem<M>) * 4; }
 
-// Rounding of a given plan for M = 64: one CTA of 4 warps per block.  The
-// 4096 keys are sorted by the whole CTA (32 per thread); greedy, repair and
-// the sweeps run on warp 0; the gain table is filled by all 128 threads.
-template <typename Key>
-union RoundCta64Work {
-    Key xbuf[4096];                 // sort exchange between warps
-    RoundShared<64> sh;             // after the sort
-};
+// ---------------------------------------------------------------------------
+// M = 64: one CTA of 4 warps per block.  The 4096 keys are sorted by the
+// whole CTA (32 per thread); greedy and repair run on warp 0; the local
+// search runs on all 128 threads (two per row) in max-plus form:
+//   B_x[j] = -a_xj for j in O_x, else -inf;  C_x[j] = a_xj for j not in O_x,
+//   else -inf;  g(x, y) = max_j (C_y[j] + B_x[j]) + max_j (C_x[j] + B_y[j]).
+// C_y[j] + B_x[j] is a_yj - a_xj exactly (IEEE a - b is a + (-b)) where j is
+// in O_x \ O_y and -inf elsewhere, so g is the same fp32 value as the
+// bit-tested form used for M <= 32, with no per-column tests.
+// ---------------------------------------------------------------------------
 
-// Steps 1-4 for one M = 64 block by a CTA of 4 warps (every thread calls it,
-// `ok` uniform over the CTA).  `key`: this thread's 32 keys; `a`: |W| with row
-// stride 65.  The final row bitmasks are in work.sh.rowbits.
-template <typename Key>
-__device__ bool round_block_cta64(Key (&key)[32], const float* a, RoundCta64Work<Key>& work, int* okflag, int N,
-                                  int sweeps, int tid) {
-    constexpr int M = 64;
-    const int lane = tid & 31, warp = tid >> 5;
-    cta_bitonic_sort64(key, work.xbuf, warp, lane);
-    __syncthreads();
+// 3-input maximum (sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// B and C rows in shared memory (row stride M floats) keep their 16-byte
+// chunks XOR-swizzled by the row index, so that threads reading chunk c of
+// different rows (the gain table setup) hit different banks: logical chunk c
+// of row r is stored at chunk c ^ (r % 16).
+template <int M>
+__device__ __forceinline__ int bc_index(int r, int j) {
+    return r * M + ((((j >> 2) ^ r) & (M / 4 - 1)) << 2) + (j & 3);
+}
+
+// max_j (u[j] + v[j]) over this thread's CPT columns (logical chunks c0 ..
+// c0 + CPT/4 - 1) of row r of a swizzled B or C array.
+template <int M, int CPT>
+__device__ __forceinline__ float max_plus(const float (&u)[CPT], const float* arr, int r, int c0) {
+    float t0 = -INFINITY, t1 = -INFINITY;
+    const float* row = arr + r * M;
 #pragma unroll
-    for (int r = 0; r < 32; ++r) work.sh.order[tid * 32 + r] = static_cast<uint16_t>(key[r].index());
-    __syncthreads();
-    if (warp == 0) {
-        const bool g = greedy_and_repair<M, 4096>(a, work.sh, N, lane);
-        if (lane == 0) *okflag = g;
+    for (int q = 0; q < CPT / 4; ++q) {
+        const float4 w = *reinterpret_cast<const float4*>(row + ((((c0 + q) ^ r) & (M / 4 - 1)) << 2));
+        const float2 s0 = add2(make_float2(u[4 * q], u[4 * q + 1]), make_float2(w.x, w.y));
+        const float2 s1 = add2(make_float2(u[4 * q + 2], u[4 * q + 3]), make_float2(w.z, w.w));
+        t0 = max3f(t0, s0.x, s0.y);
+        t1 = max3f(t1, s1.x, s1.y);
+    }
+    return fmaxf(t0, t1);
+}
+
+// Best partner of row x (lowest partner index on ties) by the two threads of
+// row x, each scanning half of the cached gains; both threads must call it.
+template <int M>
+__device__ __forceinline__ void rescan_row_pair(const RoundView<M>& sh, int x, int h, int lane) {
+    constexpr int GS = M + 1, HALF = M / 2;
+    float g[HALF];
+#pragma unroll
+    for (int k = 0; k < HALF; ++k) g[k] = sh.G[x * GS + h * HALF + k];
+    float bv = -INFINITY;
+    int bp = -1;
+#pragma unroll
+    for (int k = 0; k < HALF; ++k) {
+        const int y = h * HALF + k;
+        if (y == x) continue;
+        if (bp < 0 || g[k] > bv) { bv = g[k]; bp = y; }
+    }
+    const unsigned pair = 3u << (lane & 30);
+    const float ov = __shfl_xor_sync(pair, bv, 1);
+    const int op = __shfl_xor_sync(pair, bp, 1);
+    // the lower half's candidate wins ties (lower partner index)
+    if (h == 0 ? (ov > bv) : !(bv > ov)) { bv = ov; bp = op; }
+    if (h == 0) {
+        sh.bestv[x] = bv;
+        sh.bestp[x] = bp;
+    }
+}
+
+// Step 4 for one M = 64 block by 128 threads.  `a`: |W| (row stride M+1),
+// read only until the B/C arrays are built; sh.G may overlay it.  Bm, Cm:
+// M x M floats each (swizzled rows, bc_index), 16-byte aligned.
+template <int M>
+__device__ void local_search_mp(const float* a, float* Bm, float* Cm, const RoundView<M>& sh, int sweeps, int tid) {
+    using L = LsCfg<M>;
+    using Bits = typename WarpRound<M>::Bits;
+    constexpr int AS = M + 1, GS = M + 1, CH = L::CH, CPT = L::CPT;
+    static_assert(L::NT == 2 * M && CH == 2, "two threads per row");
+    const int lane = tid & 31;
+    const int y = tid / CH, h = tid % CH, j0 = h * CPT;
+    float By[CPT], Cy[CPT];                          // this thread's columns of B_y and C_y
+    {
+        const Bits Oy = sh.rowbits[y];
+#pragma unroll
+        for (int jj = 0; jj < CPT; ++jj) {
+            const float v = a[y * AS + j0 + jj];
+            const bool in = (Oy >> (j0 + jj)) & 1;
+            By[jj] = in ? -v : -INFINITY;
+            Cy[jj] = in ? -INFINITY : v;
+        }
+#pragma unroll
+        for (int q = 0; q < CPT / 4; ++q) {
+            const int e = bc_index<M>(y, j0 + 4 * q);
+            *reinterpret_cast<float4*>(Bm + e) = make_float4(By[4 * q], By[4 * q + 1], By[4 * q + 2], By[4 * q + 3]);
+            *reinterpret_cast<float4*>(Cm + e) = make_float4(Cy[4 * q], Cy[4 * q + 1], Cy[4 * q + 2], Cy[4 * q + 3]);
+        }
+    }
+    __syncthreads();                                 // B, C complete; |W| is not read again (G may overlay it)
+
+    // gain table: row y with rows y+1 .. y+M/2 (mod M), every unordered pair once
+#pragma unroll 1
+    for (int d = 1; d <= M / 2; ++d) {
+        const int x = (y + d) & (M - 1);
+        const float txy = row_max<CH>(max_plus<M, CPT>(Cy, Bm, x, j0 / 4));   // j in O_x \ O_y: a_yj - a_xj
+        const float tyx = row_max<CH>(max_plus<M, CPT>(By, Cm, x, j0 / 4));   // j in O_y \ O_x: a_xj - a_yj
+        if (h == 0 && !(d == M / 2 && y >= M / 2)) {
+            const float g = __fadd_rn(txy, tyx);
+            sh.G[x * GS + y] = g;
+            sh.G[y * GS + x] = g;
+        }
     }
     __syncthreads();
-    const bool ok = *okflag;
+    rescan_row_pair<M>(sh, y, h, lane);
+    __syncthreads();
+
+    int quiet = 0;                                   // anchors in a row without a swap
+    for (int sw = 0; sw < sweeps && quiet < M; ++sw) {
+        for (int i = 0; i < M && quiet < M; ++i) {
+            const float best = sh.bestv[i];
+            const int bp = sh.bestp[i];
+            if (!(best > 0.f)) { ++quiet; continue; }
+            // entries to exchange (every warp finds the same pair): lowest index on ties
+            float v1 = -INFINITY, v2 = -INFINITY;
+            int j1 = INT_MAX, j2 = INT_MAX;
+#pragma unroll
+            for (int jj = lane; jj < M; jj += 32) {
+                const int ei = bc_index<M>(i, jj), eb = bc_index<M>(bp, jj);
+                const float d1 = Cm[eb] + Bm[ei];                      // j in O_i \ O_bp: a_bp,j - a_ij
+                if (d1 > -INFINITY && (j1 == INT_MAX || d1 > v1)) { v1 = d1; j1 = jj; }
+                const float d2 = Cm[ei] + Bm[eb];                      // j in O_bp \ O_i: a_ij - a_bp,j
+                if (d2 > -INFINITY && (j2 == INT_MAX || d2 > v2)) { v2 = d2; j2 = jj; }
+            }
+            warp_argmax(v1, j1);
+            warp_argmax(v2, j2);
+            if (j1 >= M || j2 >= M) { ++quiet; continue; }   // unreachable: a positive gain needs both sets
+            quiet = 0;
+            const Bits Oi = sh.rowbits[i], Ob = sh.rowbits[bp];
+            __syncthreads();                         // everyone has read rows i and bp
+            if (tid < 4) {
+                // j1 leaves row i for row bp, j2 leaves row bp for row i: one entry per thread
+                const int r = tid < 2 ? i : bp;
+                const int j = (tid == 0 || tid == 3) ? j1 : j2;
+                const int e = bc_index<M>(r, j);
+                const bool leaves = (tid & 1) == 0;  // (i, j1) and (bp, j2) leave their rows
+                const float b = Bm[e], c = Cm[e];
+                Bm[e] = leaves ? -INFINITY : -c;
+                Cm[e] = leaves ? -b : -INFINITY;
+            } else if (tid == 4) {
+                sh.rowbits[i] = (Oi & ~(Bits(1) << j1)) | (Bits(1) << j2);
+                sh.rowbits[bp] = (Ob & ~(Bits(1) << j2)) | (Bits(1) << j1);
+            }
+            __syncthreads();                         // rows i and bp updated
+            if (y == i || y == bp) {
+#pragma unroll
+                for (int q = 0; q < CPT / 4; ++q) {
+                    const int e = bc_index<M>(y, j0 + 4 * q);
+                    const float4 wb = *reinterpret_cast<const float4*>(Bm + e);
+                    const float4 wc = *reinterpret_cast<const float4*>(Cm + e);
+                    By[4 * q] = wb.x; By[4 * q + 1] = wb.y; By[4 * q + 2] = wb.z; By[4 * q + 3] = wb.w;
+                    Cy[4 * q] = wc.x; Cy[4 * q + 1] = wc.y; Cy[4 * q + 2] = wc.z; Cy[4 * q + 3] = wc.w;
+                }
+            }
+            // new gains g(i, y) and g(bp, y) of partner row y
+            const float t1i = row_max<CH>(max_plus<M, CPT>(Cy, Bm, i, j0 / 4));
+            const float t2i = row_max<CH>(max_plus<M, CPT>(By, Cm, i, j0 / 4));
+            const float t1b = row_max<CH>(max_plus<M, CPT>(Cy, Bm, bp, j0 / 4));
+            const float t2b = row_max<CH>(max_plus<M, CPT>(By, Cm, bp, j0 / 4));
+            const float gi = __fadd_rn(t1i, t2i), gb = __fadd_rn(t1b, t2b);
+            if (h == 0) {
+                if (y != i) { sh.G[i * GS + y] = gi; sh.G[y * GS + i] = gi; }
+                if (y != i && y != bp) { sh.G[bp * GS + y] = gb; sh.G[y * GS + bp] = gb; }
+            }
+            __syncthreads();                         // gain table and rows complete
+            const int op = sh.bestp[y];
+            if (y == i || y == bp || op == i || op == bp) {   // same for both threads of row y
+                rescan_row_pair<M>(sh, y, h, lane);
+            } else if (h == 0) {
+                float bv = sh.bestv[y];
+                int b2 = op;
+                const int c1 = i < bp ? i : bp, c2 = i < bp ? bp : i;
+                const float g1 = c1 == i ? gi : gb, g2 = c2 == i ? gi : gb;
+                if (g1 > bv || (g1 == bv && c1 < b2)) { bv = g1; b2 = c1; }
+                if (g2 > bv || (g2 == bv && c2 < b2)) { bv = g2; b2 = c2; }
+                sh.bestv[y] = bv;
+                sh.bestp[y] = b2;
+            }
+            __syncthreads();                         // row bests complete
+        }
+    }
+}
+
+// Shared memory of one M = 64 block; the arrays of successive steps overlay.
+template <typename Key>
+struct Round64Smem {
+    union {
+        Key xbuf[4096];                              // sort exchange between warps
+        struct {
+            uint16_t order[4096];                    // sorted flat indices
+            int rc[64], cc[64];
+        } gr;                                        // greedy and repair
+        float bc[2 * 64 * 64];                       // local search: B, then C (row stride 64)
+    } u;
+    float a[64 * 65];                                // |W| (row stride 65); the gain table G in the local search
+    static constexpr int kColbufFloats = 512;
+    union {
+        float colbuf[kColbufFloats];                 // Dykstra phase of the fused kernel: cross-warp column sums
+        struct {
+            unsigned long long rowbits[64];
+            float bestv[64];
+            int bestp[64];
+        } rb;
+    } v;
+    int ok;
+    __device__ __forceinline__ RoundView<64> view() {
+        return RoundView<64>{a, u.gr.order, v.rb.rowbits, v.rb.bestv, v.rb.bestp, u.gr.rc, u.gr.cc};
+    }
+};
+
+// Steps 1-4 for one M = 64 block by a CTA of 4 warps (every thread calls it;
+// the result is uniform over the CTA).  `key`: this thread's 32 keys; sm.a:
+// the block's |W|.  The final row bitmasks are in sm.v.rb.rowbits.
+template <typename Key>
+__device__ bool round_block_cta64(Key (&key)[32], Round64Smem<Key>& sm, int N, int sweeps, int tid) {
+    constexpr int M = 64;
+    const int lane = tid & 31, warp = tid >> 5;
+    const RoundView<M> sh = sm.view();
+    cta_bitonic_sort64(key, sm.u.xbuf, warp, lane);
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < 32; ++r) sh.order[tid * 32 + r] = static_cast<uint16_t>(key[r].index());
+    __syncthreads();
+    if (warp == 0) {
+        const bool g = greedy_and_repair<M, 4096>(sm.a, sh, N, lane);
+        if (lane == 0) sm.ok = g;
+    }
+    __syncthreads();
+    const bool ok = sm.ok;
     if (ok && sweeps > 0) {
-        local_search<M>(a, work.sh, sweeps, tid);
+        local_search_mp<M>(sm.a, sm.u.bc, sm.u.bc + M * M, sh, sweeps, tid);
         __syncthreads();
     }
     return ok;
 }
-
-template <typename T>
-struct RoundCta64Smem {
-    RoundCta64Work<typename KeyOf<T>::type> u;
-    float a[64 * 65];               // |W|, row stride 65
-    int ok;
-};
 
 template <typename T>
 __global__ void __launch_bounds__(128)
@@ -622,7 +842,7 @@ round_cta64_kernel(const float* __restrict__ plan, const typename T::storage* __
     constexpr int M = 64, AS = 65;
     using Key = typename KeyOf<T>::type;
     extern __shared__ __align__(16) unsigned char round64_raw[];
-    RoundCta64Smem<T>& sm = *reinterpret_cast<RoundCta64Smem<T>*>(round64_raw);
+    Round64Smem<Key>& sm = *reinterpret_cast<Round64Smem<Key>*>(round64_raw);
     const int tid = threadIdx.x;
     const int64_t b = blockIdx.x;
     if (b >= n_blocks) return;                       // uniform per CTA
@@ -642,9 +862,9 @@ round_cta64_kernel(const float* __restrict__ plan, const typename T::storage* __
         key[r] = Key::make(s, a, e);
     }
     ok = __syncthreads_and(ok);
-    if (ok) ok = round_block_cta64(key, sm.a, sm.u, &sm.ok, N, sweeps, tid);
+    if (ok) ok = round_block_cta64(key, sm, N, sweeps, tid);
     if (!ok && tid == 0) atomicAdd(&g_block_failures, 1ull);
-    write_mask_rows<M>(mask, wpr, r0, c0, sm.u.sh.rowbits, ok, tid, 128);
+    write_mask_rows<M>(mask, wpr, r0, c0, sm.v.rb.rowbits, ok, tid, 128);
 }
 
 }  // namespace tsenor

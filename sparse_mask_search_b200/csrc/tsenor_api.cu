@@ -67,7 +67,7 @@ cudaError_t launch_round(const float* plan, const void* W, int64_t rows, int64_t
         if (e != cudaSuccess) return e;
     }
     if constexpr (M == 64) {
-        constexpr size_t smem = sizeof(RoundCta64Smem<T>);
+        constexpr size_t smem = sizeof(Round64Smem<typename KeyOf<T>::type>);
         cudaError_t e = cudaFuncSetAttribute(round_cta64_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              int(smem));
         if (e != cudaSuccess) return e;
@@ -110,7 +110,7 @@ cudaError_t launch_fused(const void* W, int64_t rows, int64_t cols, int N, float
         fused_kernel16<T, EXT><<<dim3(unsigned((nb + 15) / 16)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps,
                                                                                  mask, wpr, ext);
     } else {
-        constexpr size_t smem = sizeof(Fused64Smem<T>);
+        constexpr size_t smem = sizeof(Round64Smem<typename KeyOf<T>::type>);
         e = cudaFuncSetAttribute(fused_kernel64<T, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
         fused_kernel64<T, EXT><<<dim3(unsigned(nb)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps, mask, wpr,
