@@ -73,9 +73,13 @@ def mufu_peak_tops(sm_mhz):
 
 
 def source_digest():
+    """Digest of the kernel sources (the device-code headers); a profiled
+    traffic figure is used only while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_mask_search_b200", "csrc")
     for fn in sorted(os.listdir(csrc)):
+        if not fn.endswith(".cuh"):
+            continue
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]

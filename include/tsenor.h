@@ -201,6 +201,18 @@ tsenor_status tsenor_plan_warm(const void* W, tsenor_dtype dtype, int64_t rows, 
                                float* potentials, int32_t* iters_used, float* plan_out,
                                tsenor_stream_t stream);
 
+/*
+ * tsenor_mask on an importance-score matrix instead of weights.  Layer-wise
+ * pruning methods hand the solver scores rather than |W| (the review names
+ * Wanda, SparseGPT and ALPS: "Core claim", "What carries the argument"), for
+ * example |W_ij| times the norm of input feature j.
+ *   scores: rows x cols fp32 (device, 16-byte aligned); the magnitude of each
+ *           score is used, so non-negative scores are taken as they are.
+ * Same result as tsenor_mask(scores, TSENOR_F32, ...), same errors.
+ */
+tsenor_status tsenor_mask_scores(const float* scores, int64_t rows, int64_t cols, int N, int M, float tau,
+                                 int iters, int sweeps, uint32_t* mask_out, tsenor_stream_t stream);
+
 /* Static description of a status code. */
 const char* tsenor_status_string(int status);
 

@@ -18,7 +18,7 @@ STATUS = {0: "TSENOR_OK", -1: "TSENOR_ERR_ARG", -2: "TSENOR_ERR_SHAPE", -3: "TSE
 NOALLOC_MAX_PARAMS = 16 * 1024 * 1024
 EXPORTS = ("tsenor_mask", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
            "tsenor_status_string", "tsenor_last_error", "tsenor_mask_noalloc", "tsenor_mask_safeguard",
-           "tsenor_mask_padded", "tsenor_mask_warm", "tsenor_plan_warm")
+           "tsenor_mask_padded", "tsenor_mask_warm", "tsenor_plan_warm", "tsenor_mask_scores")
 
 _lib = None
 
@@ -43,6 +43,7 @@ def lib() -> C.CDLL:
         L.tsenor_plan.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, p, p]
         L.tsenor_mask_padded.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p]
         L.tsenor_mask_safeguard.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p, p, p]
+        L.tsenor_mask_scores.argtypes = [p, i64, i64, i32, i32, f32, i32, i32, p, p]
         L.tsenor_mask_warm.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, f32, i32, p, p, p, p]
         L.tsenor_plan_warm.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, f32, i32, p, p, p, p]
         L.tsenor_round.argtypes = [p, p, i32, i64, i64, i32, i32, i32, p, p]
@@ -139,6 +140,20 @@ def tsenor_mask_safeguard(W, prev_mask, N: int, M: int, tau: float, iters: int, 
     _check(lib().tsenor_mask_safeguard(W.data_ptr(), _dtype_code(W), rows, cols, N, M, float(tau), iters, sweeps,
                                        prev_mask.data_ptr(), out.data_ptr(),
                                        kept.data_ptr() if kept is not None else None, _stream_handle(stream)))
+    return out
+
+
+def tsenor_mask_scores(scores, N: int, M: int, tau: float, iters: int, sweeps: int, out=None, stream=None):
+    """Transposable N:M mask of an importance-score matrix (float32; magnitudes are used)."""
+    import torch
+    _check_2d_cuda(scores, "scores")
+    if scores.dtype != torch.float32:
+        raise TypeError("scores must be float32")
+    rows, cols = scores.shape
+    if out is None:
+        out = torch.empty((rows, words_per_row(cols)), dtype=torch.int32, device=scores.device)
+    _check(lib().tsenor_mask_scores(scores.data_ptr(), rows, cols, N, M, float(tau), iters, sweeps, out.data_ptr(),
+                                    _stream_handle(stream)))
     return out
 
 
@@ -258,6 +273,6 @@ def tsenor_error_count(stream=None) -> int:
     return int(n.value)
 
 
-__all__ = ["tsenor_mask", "tsenor_mask_noalloc", "tsenor_mask_safeguard", "tsenor_mask_padded", "tsenor_mask_warm",
+__all__ = ["tsenor_mask", "tsenor_mask_scores", "tsenor_mask_noalloc", "tsenor_mask_safeguard", "tsenor_mask_padded", "tsenor_mask_warm",
            "tsenor_plan", "tsenor_plan_warm", "tsenor_round", "tsenor_objective", "tsenor_error_count",
            "TsenorError", "lib", "words_per_row", "EXPORTS", "LIB_PATH"]

@@ -246,6 +246,11 @@ extern "C" tsenor_status tsenor_mask(const void* W, tsenor_dtype dtype, int64_t 
     return TSENOR_OK;
 }
 
+extern "C" tsenor_status tsenor_mask_scores(const float* scores, int64_t rows, int64_t cols, int N, int M, float tau,
+                                            int iters, int sweeps, uint32_t* mask_out, tsenor_stream_t stream) {
+    return tsenor_mask(scores, TSENOR_F32, rows, cols, N, M, tau, iters, sweeps, mask_out, stream);
+}
+
 extern "C" tsenor_status tsenor_mask_warm(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols, int N,
                                           int M, float tau, int iters, int sweeps, float tol, int warm,
                                           float* potentials, int32_t* iters_used, uint32_t* mask_out,

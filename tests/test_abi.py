@@ -95,6 +95,13 @@ def test_warm_entry_points_validate(kw, code):
                                   a["warm"], a["pot"], a["used"], a["out"], None) == code
 
 
+def test_scores_entry_point_validates():
+    L = tsl.lib()
+    assert L.tsenor_mask_scores(1 << 12, 64, 64, 2, 4, 10.0, 5, 1, 0, None) == -1          # no mask buffer
+    assert L.tsenor_mask_scores(1 << 12, 64, 62, 2, 4, 10.0, 5, 1, 1 << 12, None) == -2
+    assert L.tsenor_mask_scores(0, 0, 64, 2, 4, 10.0, 5, 1, 0, None) == 0                   # empty
+
+
 def test_warm_empty_calls_do_nothing():
     L = tsl.lib()
     assert _warm(L, rows=0, W=0, out=0, pot=0, used=0) == 0

@@ -23,7 +23,9 @@ def test_wanda_style_scores(M, N):
     _, W = synth.make_matrix(rows, cols, "f32", "normal", 0.02, seed=M)
     xnorm = 0.5 + synth.rng(100 + M).random(cols).astype(np.float32)       # input feature norms
     scores = (np.abs(W) * xnorm[None, :]).astype(np.float32)
-    m = mask_to_np(tsl.tsenor_mask(to_device(scores, "f32"), N, M, 20.0, 200, 4))
+    sd = to_device(scores, "f32")
+    m = mask_to_np(tsl.tsenor_mask_scores(sd, N, M, 20.0, 200, 4))
+    assert (m == mask_to_np(tsl.tsenor_mask(sd, N, M, 20.0, 200, 4))).all()
     m_ref, _, _ = oracle.mask(scores, N, M, 20.0, 200, 4)
     bg, br = block_bits(m, cols, M), block_bits(m_ref, cols, M)
     assert (bg.sum(axis=3) == N).all() and (bg.sum(axis=2) == N).all()
