@@ -69,6 +69,10 @@ struct F32 {
         out[0] = fabsf(v.x); out[1] = fabsf(v.y); out[2] = fabsf(v.z); out[3] = fabsf(v.w);
     }
     __device__ __forceinline__ static float load1(const float* p) { return fabsf(__ldg(p)); }
+    __device__ __forceinline__ static void smem16(const float* p, float* out) {     // 16 bytes of shared memory
+        const float4 v = *reinterpret_cast<const float4*>(p);
+        out[0] = fabsf(v.x); out[1] = fabsf(v.y); out[2] = fabsf(v.z); out[3] = fabsf(v.w);
+    }
 };
 
 struct BF16 {
@@ -87,6 +91,15 @@ struct BF16 {
         }
     }
     __device__ __forceinline__ static float load1(const uint16_t* p) { return widen(__ldg(p)); }
+    __device__ __forceinline__ static void smem16(const uint16_t* p, float* out) {  // 16 bytes of shared memory
+        const uint4 v = *reinterpret_cast<const uint4*>(p);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            out[2 * q] = widen(w[q] & 0xffffu);
+            out[2 * q + 1] = widen(w[q] >> 16);
+        }
+    }
 };
 
 // Packed sort key of one block entry: plan bits (S >= 0, so the bit pattern

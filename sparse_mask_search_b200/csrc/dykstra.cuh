@@ -28,6 +28,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "tma.cuh"
 
 namespace tsenor {
 
@@ -228,27 +229,77 @@ struct TileThread {
 // Dykstra for one block spread over its TPB threads.  On return `y` holds the
 // final state of this thread's sub-tile and `tile` the block's |W| (M x M in
 // shared memory, row stride TS).  Contains CTA-wide barriers: every thread of the CTA
-// must call it.  Returns whether the block's W is finite.
+// must call it.  Returns whether the block's W is finite (false too when its
+// tile copy did not complete in time).
+// Where a block's W tile comes from.  With a tensor map (`map` non-null) the
+// tile (rows r0.., columns c0..) is copied by TMA into `raw` (M*M elements,
+// 128-byte aligned, shared memory) on the barrier `bar` and then widened to
+// |W|; otherwise the block's threads read it from `W` (row stride `cols`)
+// with 16-byte loads.
+template <typename T>
+struct TileSource {
+    const CUtensorMap* map;
+    typename T::storage* raw;
+    uint64_t* bar;
+    const typename T::storage* W;
+    int64_t cols;
+};
+
 // EXT: warm start from / export to ext.potentials of block b, stop rule
 // ext.tol2, iteration count to ext.iters_used.
 template <int M, typename T, int TS = M, bool EXT = false>
-__device__ __forceinline__ bool dykstra_tile_solve(const typename T::storage* __restrict__ W, int64_t cols,
-                                                   int64_t r0, int64_t c0, bool active, int N, float tau,
-                                                   int iters, float* tile, float* colbuf,
+__device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int64_t r0, int64_t c0, bool active,
+                                                   int N, float tau, int iters, float* tile, float* colbuf,
                                                    const TileThread<M>& th, float (&y)[4][8],
                                                    const DykstraExt& ext = DykstraExt{}, int64_t b = 0) {
     using C = TileCfg<M>;
     constexpr int P = C::P, Q = C::Q;
     const int lane = th.lane, warp = th.warp;
 
-    // ---- stage |W| of the block in shared memory (16-byte coalesced loads)
-    {
+    bool loaded = true;
+    if (!src.map) {
+        // ---- 16-byte loads of the block's tile straight into |W|
         constexpr int V = T::kVec;
         constexpr int CPR = M / V;                 // 16-byte chunks per tile row
         for (int q = th.t; q < M * CPR; q += C::TPB) {
             const int i = q / CPR, v = q % CPR;
             float tmp[V];
-            if (active) T::load16(W + (r0 + i) * cols + c0 + v * V, tmp);
+            if (active) T::load16(src.W + (r0 + i) * src.cols + c0 + v * V, tmp);
+            else {
+#pragma unroll
+                for (int u = 0; u < V; ++u) tmp[u] = 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < V; ++u) tile[i * TS + v * V + u] = tmp[u];
+        }
+    } else {
+        // ---- stage the block's W tile in shared memory by TMA, then |W| into the tile
+        typename T::storage* raw = src.raw;
+        uint64_t* bar = src.bar;
+        const CUtensorMap* wmap = src.map;
+        // a staging address off the 128-byte grid is never handed to the copy
+        // engine: the block is reported as failed instead
+        const bool staged = (smem_u32(raw) & 127u) == 0 && (smem_u32(bar) & 7u) == 0;
+        if (active && staged && th.t == 0) {
+            mbar_init(bar, 1);
+            mbar_init_fence();
+        }
+        if constexpr (C::TPB <= 32) __syncwarp(); else __syncthreads();   // barrier initialised before any poll
+        if (active && staged && th.t == 0) {
+            mbar_arrive_expect_tx(bar, unsigned(M * M * sizeof(typename T::storage)));
+            tma_load_2d(raw, wmap, int(c0), int(r0), bar);
+        }
+        if (active) {
+            loaded = staged && mbar_wait_bounded(bar, 0);
+            // a copy that did not land in time may still arrive: wait once more before the space is reused
+            if (staged && !loaded) mbar_wait_bounded(bar, 0);
+        }
+        constexpr int V = 16 / int(sizeof(typename T::storage));   // elements per 16-byte chunk
+        constexpr int CPR = M / V;                                  // chunks per tile row
+        for (int q = th.t; q < M * CPR; q += C::TPB) {
+            const int i = q / CPR, v = q % CPR;
+            float tmp[V];
+            if (active && loaded) T::smem16(raw + i * M + v * V, tmp);
             else {
 #pragma unroll
                 for (int u = 0; u < V; ++u) tmp[u] = 0.f;
@@ -260,7 +311,7 @@ __device__ __forceinline__ bool dykstra_tile_solve(const typename T::storage* __
     __syncthreads();
 
     float m = 0.f;
-    bool finite = true;
+    bool finite = loaded;
 #pragma unroll
     for (int k = 0; k < P; ++k)
 #pragma unroll
@@ -491,23 +542,39 @@ __device__ __forceinline__ bool dykstra_tile_solve(const typename T::storage* __
     return finite;
 }
 
+// Shared memory of dykstra_tile_kernel: TMA staging of the raw W tiles, the
+// |W| tiles, the cross-warp column buffer, one barrier per block slot.
+template <int M, typename T>
+struct PlanSmem {
+    using C = TileCfg<M>;
+    static constexpr size_t raw_bytes = size_t(C::BPC) * M * M * sizeof(typename T::storage);
+    static constexpr size_t tile_off = (raw_bytes + 127) / 128 * 128;
+    static constexpr size_t colbuf_off = tile_off + sizeof(float) * C::BPC * M * M;
+    static constexpr size_t bar_off = colbuf_off + sizeof(float) * (C::WC > 1 ? 2 * 4 * 32 * C::CO : 0);
+    static constexpr size_t bytes = bar_off + sizeof(uint64_t) * C::BPC;
+};
+
 template <int M, typename T, bool EXT = false>
 __global__ void __launch_bounds__(128)
-dykstra_tile_kernel(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks,
+dykstra_tile_kernel(const __grid_constant__ CUtensorMap wmap, int64_t cols, int64_t n_blocks,
                     int N, float tau, int iters, float* __restrict__ plan, DykstraExt ext = {}) {
     using C = TileCfg<M>;
-    extern __shared__ float smem[];
+    using L = PlanSmem<M, T>;
+    extern __shared__ __align__(128) unsigned char plan_raw[];
     const TileThread<M> th;
-    float* tile = smem + th.blk * M * M;
-    float* colbuf = smem + C::BPC * M * M;         // [2][warps][32][CO] for cross-warp columns
+    auto* raw = reinterpret_cast<typename T::storage*>(plan_raw) + th.blk * M * M;
+    float* tile = reinterpret_cast<float*>(plan_raw + L::tile_off) + th.blk * M * M;
+    float* colbuf = reinterpret_cast<float*>(plan_raw + L::colbuf_off);   // [2][warps][32][CO]
+    uint64_t* bar = reinterpret_cast<uint64_t*>(plan_raw + L::bar_off) + th.blk;
     const int64_t b = int64_t(blockIdx.x) * C::BPC + th.blk;
     const bool active = b < n_blocks;
     const int64_t nbc = cols / M;
     const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
 
     float y[C::P][C::Q];
-    const bool finite = dykstra_tile_solve<M, T, M, EXT>(W, cols, r0, c0, active, N, tau, iters, tile, colbuf, th, y,
-                                                         ext, b);
+    const TileSource<T> src{&wmap, raw, bar, nullptr, 0};
+    const bool finite = dykstra_tile_solve<M, T, M, EXT>(src, r0, c0, active, N, tau, iters, tile, colbuf, th, y, ext,
+                                                         b);
 
     // ---- plan via the smem tile, then 16-byte coalesced stores
     __syncthreads();
@@ -527,10 +594,7 @@ dykstra_tile_kernel(const typename T::storage* __restrict__ W, int64_t cols, int
     }
 }
 
-template <int M>
-constexpr size_t dykstra_tile_smem() {
-    using C = TileCfg<M>;
-    return sizeof(float) * (C::BPC * M * M + (C::WC > 1 ? 2 * 4 * 32 * C::CO : 0));
-}
+template <int M, typename T>
+constexpr size_t dykstra_tile_smem() { return PlanSmem<M, T>::bytes; }
 
 }  // namespace tsenor

@@ -8,7 +8,7 @@
 //  - M = 64: one CTA of 4 warps per block; the CTA sorts, warp 0 runs the
 //    greedy and the repair, all 128 threads the local search.
 // EXT instances add the warm start, the stop rule and the potentials export
-// of dykstra_tile_solve.
+// of dykstra_tile_solve.  M = 16 and 64 stage the W tiles by TMA.
 #pragma once
 
 #include <type_traits>
@@ -20,6 +20,9 @@ namespace tsenor {
 
 // bf16: registers capped for 5 CTAs (20 warps) per SM (5.00 ms against 5.03 ms
 // uncapped on the 4096x11008 16:32 workload); the fp32 key needs more.
+// The tile is read with 16-byte loads here, not staged by TMA: on the same
+// workload the TMA-staged variant of this kernel timed 5.16 ms against
+// 5.01 ms (the plan kernel of the same M gained 0.7% from TMA staging).
 template <typename T, bool EXT = false>
 __global__ void __launch_bounds__(128, std::is_same<T, BF16>::value ? 5 : 4)
 fused_kernel32(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
@@ -29,18 +32,19 @@ fused_kernel32(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
     using Key = typename KeyOf<T>::type;
     static_assert(C::TPB == 32 && C::BPC == 4, "one warp per block");
     constexpr int TS = M + 1;                       // tile row stride (conflict-free column access)
-    extern __shared__ float fused_smem[];
+    extern __shared__ __align__(16) unsigned char fused32_raw[];
     const TileThread<M> th;
-    float* tile = fused_smem + th.blk * M * TS;
-    RoundShared<M>* shs = reinterpret_cast<RoundShared<M>*>(fused_smem + C::BPC * M * TS);
+    float* tile = reinterpret_cast<float*>(fused32_raw) + th.blk * M * TS;
+    RoundShared<M>* shs = reinterpret_cast<RoundShared<M>*>(reinterpret_cast<float*>(fused32_raw) + C::BPC * M * TS);
     const int64_t b = int64_t(blockIdx.x) * C::BPC + th.blk;
     const bool active = b < n_blocks;
     const int64_t nbc = cols / M;
     const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
 
     float y[C::P][C::Q];
-    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(W, cols, r0, c0, active, N, tau, iters, tile, nullptr, th,
-                                                          y, ext, b);
+    const TileSource<T> src{nullptr, nullptr, nullptr, W, cols};
+    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(src, r0, c0, active, N, tau, iters, tile, nullptr, th, y,
+                                                          ext, b);
     if (!active) return;                              // no CTA-wide barrier follows
 
     Key key[C::P * C::Q];
@@ -65,18 +69,20 @@ constexpr size_t fused32_smem() {
 // M = 16: a warp holds 4 blocks of 8 threads each.
 template <typename T, bool EXT = false>
 __global__ void __launch_bounds__(128)
-fused_kernel16(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
+fused_kernel16(const __grid_constant__ CUtensorMap wmap, int64_t cols, int64_t n_blocks, int N, float tau,
                int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr, DykstraExt ext = {}) {
     constexpr int M = 16, TS = M + 1, E = M * M;
     using C = TileCfg<M>;
     using Key = typename KeyOf<T>::type;
     constexpr int BPW = C::BPW, R = WarpRound<M>::R;
     static_assert(C::TPB == 8 && BPW == 4 && C::BPC == 16, "four blocks per warp");
-    extern __shared__ float fused_smem[];
-    float* atiles = fused_smem;                               // [BPC][M * TS] |W|
-    float* ptiles = atiles + C::BPC * M * TS;                 // [BPC][M * M]  plan
+    static_assert((C::BPC * M * TS * 4) % 128 == 0 && (E * 4) % 128 == 0, "TMA staging alignment");
+    extern __shared__ __align__(128) unsigned char fused16_raw[];
+    float* atiles = reinterpret_cast<float*>(fused16_raw);   // [BPC][M * TS] |W|
+    float* ptiles = atiles + C::BPC * M * TS;                 // [BPC][M * M]  plan (first: TMA staging of W)
     RoundShared<M>* shs = reinterpret_cast<RoundShared<M>*>(ptiles + C::BPC * E);   // one per warp
     int* flags = reinterpret_cast<int*>(shs + 4);             // [BPC] finite
+    uint64_t* bars = reinterpret_cast<uint64_t*>(flags + C::BPC);
     const TileThread<M> th;
     float* tile = atiles + th.blk * M * TS;
     const int64_t b = int64_t(blockIdx.x) * C::BPC + th.blk;
@@ -85,8 +91,10 @@ fused_kernel16(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
     const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
 
     float y[C::P][C::Q];
-    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(W, cols, r0, c0, active, N, tau, iters, tile, nullptr, th,
-                                                          y, ext, b);
+    const TileSource<T> src{&wmap, reinterpret_cast<typename T::storage*>(ptiles + th.blk * E), bars + th.blk,
+                            nullptr, 0};
+    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(src, r0, c0, active, N, tau, iters, tile, nullptr, th, y,
+                                                          ext, b);
     float* ptile = ptiles + th.blk * E;
 #pragma unroll
     for (int k = 0; k < C::P; ++k)
@@ -119,8 +127,11 @@ fused_kernel16(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
 }
 
 constexpr size_t fused16_smem() {
-    return sizeof(float) * 16 * (16 * 17 + 16 * 16) + sizeof(RoundShared<16>) * 4 + sizeof(int) * 16;
+    return sizeof(float) * 16 * (16 * 17 + 16 * 16) + sizeof(RoundShared<16>) * 4 + sizeof(int) * 16 +
+           sizeof(uint64_t) * 16;
 }
+static_assert((sizeof(float) * 16 * (16 * 17 + 16 * 16) + sizeof(RoundShared<16>) * 4 + sizeof(int) * 16) % 8 == 0,
+              "barrier alignment");
 
 // M = 64: one CTA of 4 warps per block; Round64Smem's colbuf serves the
 // Dykstra phase's cross-warp column sums.
@@ -128,13 +139,14 @@ static_assert(Round64Smem<KeyB>::kColbufFloats >= 2 * 4 * 32 * TileCfg<64>::CO, 
 
 template <typename T, bool EXT = false>
 __global__ void __launch_bounds__(128)
-fused_kernel64(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
+fused_kernel64(const __grid_constant__ CUtensorMap wmap, int64_t cols, int64_t n_blocks, int N, float tau,
                int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr, DykstraExt ext = {}) {
     constexpr int M = 64, TS = M + 1;
     using C = TileCfg<M>;
     using Key = typename KeyOf<T>::type;
     static_assert(C::TPB == 128 && C::BPC == 1, "one block per CTA");
-    extern __shared__ __align__(16) unsigned char fused64_raw[];
+    static_assert(sizeof(Round64Smem<Key>::u) >= M * M * sizeof(typename T::storage), "TMA staging size");
+    extern __shared__ __align__(128) unsigned char fused64_raw[];
     Round64Smem<Key>& sm = *reinterpret_cast<Round64Smem<Key>*>(fused64_raw);
     const TileThread<M> th;
     const int64_t b = blockIdx.x;
@@ -143,8 +155,10 @@ fused_kernel64(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
     const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
 
     float y[C::P][C::Q];
-    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(W, cols, r0, c0, true, N, tau, iters, sm.a, sm.v.colbuf,
-                                                          th, y, ext, b);
+    // the raw W tile is staged in the sort exchange space
+    const TileSource<T> src{&wmap, reinterpret_cast<typename T::storage*>(&sm.u), &sm.tma_bar, nullptr, 0};
+    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(src, r0, c0, true, N, tau, iters, sm.a, sm.v.colbuf, th, y,
+                                                          ext, b);
     Key key[C::P * C::Q];
 #pragma unroll
     for (int k = 0; k < C::P; ++k)

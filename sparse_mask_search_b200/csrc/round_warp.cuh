@@ -804,6 +804,7 @@ struct Round64Smem {
         } rb;
     } v;
     int ok;
+    uint64_t tma_bar;                                // fused kernel: completion of the W tile copy
     __device__ __forceinline__ RoundView<64> view() {
         return RoundView<64>{a, u.gr.order, v.rb.rowbits, v.rb.bestv, v.rb.bestp, u.gr.rc, u.gr.cc};
     }

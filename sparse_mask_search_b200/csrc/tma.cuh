@@ -1,0 +1,62 @@
+// Tensor-memory-accelerator (TMA) staging of W tiles into shared memory:
+// one elected thread per block issues a 2D bulk tensor copy of the block's
+// M x M tile (cp.async.bulk.tensor, no multicast) that completes on an
+// mbarrier; the block's threads wait on the barrier with a bounded number of
+// polls.  The tensor map is encoded on the host for each call.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace tsenor {
+
+__device__ __forceinline__ unsigned smem_u32(const void* p) {
+    return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Makes an initialised barrier visible to the asynchronous (TMA) proxy.
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+    unsigned done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Polls until the barrier's phase `parity` completes, at most kTmaPolls times
+// (each poll may suspend the thread for a short hardware-defined time).
+constexpr unsigned kTmaPolls = 1u << 18;
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity) {
+    for (unsigned k = 0; k < kTmaPolls; ++k)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// 2D tile load: box origin (x = column, y = row) of the tensor map into
+// shared memory at dst (128-byte aligned); completion is counted in bytes on
+// `bar`.  x * element size is a multiple of 16 for every call in this library.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+}  // namespace tsenor

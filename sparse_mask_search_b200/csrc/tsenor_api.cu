@@ -5,6 +5,8 @@
 #include <mutex>
 #include <type_traits>
 
+#include <cudaTypedefs.h>
+
 #include "../../include/tsenor.h"
 #include "common.cuh"
 #include "dykstra.cuh"
@@ -36,6 +38,35 @@ tsenor_status check_common(const void* W, int dtype, int64_t rows, int64_t cols,
 }
 
 // EXT = warm start / stop rule / potentials export (tsenor_mask_warm, tsenor_plan_warm).
+// Tensor map of W for the TMA tile copies: a rows x cols row-major matrix of
+// T::storage, box M x M.  cuTensorMapEncodeTiled is fetched from the driver
+// once (no link against the driver library).
+PFN_cuTensorMapEncodeTiled g_encode_tiled = nullptr;
+std::once_flag g_encode_once;
+
+template <typename T>
+cudaError_t encode_w_map(CUtensorMap* map, const void* W, int64_t rows, int64_t cols, int M) {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
+    });
+    if (!g_encode_tiled) return cudaErrorNotSupported;
+    constexpr size_t es = sizeof(typename T::storage);
+    const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(cols) * es};          // bytes, a multiple of 16 (cols % 16 == 0)
+    const cuuint32_t box[2] = {cuuint32_t(M), cuuint32_t(M)};       // inner box M * es bytes, a multiple of 16
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapDataType dt = std::is_same<T, BF16>::value ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                                : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUresult r = g_encode_tiled(map, dt, 2, const_cast<void*>(W), dims, strides, box, estr,
+                                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int M, typename T, bool EXT>
 cudaError_t launch_plan(const void* W, int64_t rows, int64_t cols, int N, float tau, int iters,
                         float* plan, cudaStream_t st, const DykstraExt& ext) {
@@ -45,13 +76,16 @@ cudaError_t launch_plan(const void* W, int64_t rows, int64_t cols, int N, float 
         const int64_t grid = (nb + 127) / 128;
         dykstra_thread_kernel<M, T, EXT><<<dim3(unsigned(grid)), 128, 0, st>>>(w, cols, nb, N, tau, iters, plan, ext);
     } else {
-        constexpr size_t smem = dykstra_tile_smem<M>();
-        cudaError_t e = cudaFuncSetAttribute(dykstra_tile_kernel<M, T, EXT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        CUtensorMap map;
+        cudaError_t e = encode_w_map<T>(&map, W, rows, cols, M);
+        if (e != cudaSuccess) return e;
+        constexpr size_t smem = dykstra_tile_smem<M, T>();
+        e = cudaFuncSetAttribute(dykstra_tile_kernel<M, T, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem));
         if (e != cudaSuccess) return e;
         const int64_t grid = (nb + TileCfg<M>::BPC - 1) / TileCfg<M>::BPC;
         dykstra_tile_kernel<M, T, EXT><<<dim3(unsigned(grid)), TileCfg<M>::THREADS, smem, st>>>(
-            w, cols, nb, N, tau, iters, plan, ext);
+            map, cols, nb, N, tau, iters, plan, ext);
     }
     return cudaGetLastError();
 }
@@ -91,15 +125,18 @@ cudaError_t launch_fused(const void* W, int64_t rows, int64_t cols, int N, float
                          uint32_t* mask, cudaStream_t st, const DykstraExt& ext) {
     const int64_t nb = (rows / M) * (cols / M);
     const int64_t wpr = (cols + 31) / 32;
-    const auto* w = static_cast<const typename T::storage*>(W);
     cudaError_t e = cudaSuccess;
     if constexpr (M == 32) {
+        const auto* w = static_cast<const typename T::storage*>(W);
         constexpr size_t smem = fused32_smem();
         e = cudaFuncSetAttribute(fused_kernel32<T, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
         fused_kernel32<T, EXT><<<dim3(unsigned((nb + 3) / 4)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps,
                                                                                mask, wpr, ext);
     } else if constexpr (M == 16) {
+        CUtensorMap w;
+        e = encode_w_map<T>(&w, W, rows, cols, M);
+        if (e != cudaSuccess) return e;
         if (cols % 32) {
             e = cudaMemsetAsync(mask, 0, size_t(rows) * size_t(wpr) * 4, st);   // padding bits
             if (e != cudaSuccess) return e;
@@ -110,6 +147,9 @@ cudaError_t launch_fused(const void* W, int64_t rows, int64_t cols, int N, float
         fused_kernel16<T, EXT><<<dim3(unsigned((nb + 15) / 16)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps,
                                                                                  mask, wpr, ext);
     } else {
+        CUtensorMap w;
+        e = encode_w_map<T>(&w, W, rows, cols, M);
+        if (e != cudaSuccess) return e;
         constexpr size_t smem = sizeof(Round64Smem<typename KeyOf<T>::type>);
         e = cudaFuncSetAttribute(fused_kernel64<T, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
