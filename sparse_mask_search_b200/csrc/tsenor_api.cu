@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "dykstra.cuh"
 #include "round_warp.cuh"
+#include "round_group.cuh"
 #include "fused.cuh"
 #include "objective.cuh"
 
@@ -100,7 +101,15 @@ cudaError_t launch_round(const float* plan, const void* W, int64_t rows, int64_t
         cudaError_t e = cudaMemsetAsync(mask, 0, size_t(rows) * size_t(wpr) * 4, st);
         if (e != cudaSuccess) return e;
     }
-    if constexpr (M == 64) {
+    if constexpr (M <= 8) {
+        constexpr size_t smem = round_group_smem<M>();
+        constexpr int64_t bpc = 4 * GroupRound<M>::BPW;
+        cudaError_t e = cudaFuncSetAttribute(round_group_kernel<M, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(smem));
+        if (e != cudaSuccess) return e;
+        round_group_kernel<M, T><<<dim3(unsigned((nb + bpc - 1) / bpc)), 128, smem, st>>>(
+            plan, static_cast<const typename T::storage*>(W), cols, nb, N, sweeps, mask, wpr);
+    } else if constexpr (M == 64) {
         constexpr size_t smem = sizeof(Round64Smem<typename KeyOf<T>::type>);
         cudaError_t e = cudaFuncSetAttribute(round_cta64_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              int(smem));
