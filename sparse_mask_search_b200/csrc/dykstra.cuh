@@ -109,35 +109,49 @@ dykstra_thread_kernel(const typename T::storage* __restrict__ W, int64_t cols, i
             for (int j = 0; j < M; ++j) y[i][j] += float(U[i] + V[j]);
     }
 
+    // column pairs (j, j+1) as packed fp32x2 values
+    constexpr int M2 = M / 2;
+    float2 y2[M][M2];
+#pragma unroll
+    for (int i = 0; i < M; ++i)
+#pragma unroll
+        for (int c = 0; c < M2; ++c) y2[i][c] = make_float2(y[i][2 * c], y[i][2 * c + 1]);
     if (finite) {
         for (int t = 0; t < iters; ++t) {
             float delta = 0.f;                         // largest |r_i|, |c_j| of this iteration (EXT)
-            float C[M];
+            float2 C2[M2];
 #pragma unroll
-            for (int j = 0; j < M; ++j) C[j] = 0.f;
+            for (int c = 0; c < M2; ++c) C2[c] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < M; ++i) {
-                float e[M], R = 0.f;
+                float2 e2[M2];
 #pragma unroll
-                for (int j = 0; j < M; ++j) {
-                    e[j] = ex2(fminf(y[i][j], 0.f));
-                    R += e[j];
-                }
+                for (int c = 0; c < M2; ++c)
+                    e2[c] = make_float2(ex2(fminf(y2[i][c].x, 0.f)), ex2(fminf(y2[i][c].y, 0.f)));
+                float2 acc = e2[0];
+#pragma unroll
+                for (int c = 1; c < M2; ++c) acc = add2(acc, e2[c]);
+                const float R = acc.x + acc.y;
                 const float w = fN * rcp_newton(R);
                 const float r = log2N - lg2(R);
+                const float2 w2 = make_float2(w, w), r2 = make_float2(r, r);
 #pragma unroll
-                for (int j = 0; j < M; ++j) {
-                    C[j] = fmaf(e[j], w, C[j]);
-                    y[i][j] += r;
+                for (int c = 0; c < M2; ++c) {
+                    C2[c] = fma2(e2[c], w2, C2[c]);
+                    y2[i][c] = add2(y2[i][c], r2);
                 }
                 if constexpr (EXT) { U[i] += double(r); delta = fmaxf(delta, fabsf(r)); }
             }
 #pragma unroll
-            for (int j = 0; j < M; ++j) {
-                const float c = log2N - lg2(C[j]);
+            for (int c = 0; c < M2; ++c) {
+                const float2 cv = make_float2(log2N - lg2(C2[c].x), log2N - lg2(C2[c].y));
 #pragma unroll
-                for (int i = 0; i < M; ++i) y[i][j] += c;
-                if constexpr (EXT) { V[j] += double(c); delta = fmaxf(delta, fabsf(c)); }
+                for (int i = 0; i < M; ++i) y2[i][c] = add2(y2[i][c], cv);
+                if constexpr (EXT) {
+                    V[2 * c] += double(cv.x);
+                    V[2 * c + 1] += double(cv.y);
+                    delta = fmaxf(delta, fmaxf(fabsf(cv.x), fabsf(cv.y)));
+                }
             }
             used = t + 1;
             if constexpr (EXT) {
@@ -145,6 +159,13 @@ dykstra_thread_kernel(const typename T::storage* __restrict__ W, int64_t cols, i
             }
         }
     }
+#pragma unroll
+    for (int i = 0; i < M; ++i)
+#pragma unroll
+        for (int c = 0; c < M2; ++c) {
+            y[i][2 * c] = y2[i][c].x;
+            y[i][2 * c + 1] = y2[i][c].y;
+        }
     if constexpr (EXT) {
         if (ext.potentials) {
             float* uv = ext.potentials + 2 * M * b;
