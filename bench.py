@@ -32,6 +32,7 @@ import numpy as np  # noqa: E402
 import synth  # noqa: E402
 
 DEFAULT_WORKLOAD = "w4096x11008_bf16_t3_16of32"
+METRIC = "transposable N:M mask Gparams/s at 1 B200 (% of roofline); mean gap to exact opt"
 STACK = "stack7b"                  # 32 layers x 7 matrices, 4:8, one pass = one step
 SM_COUNT = 148
 MUFU_PER_CLK_PER_SM = 16          # ex2 / lg2 / rcp results per clock per SM
@@ -255,7 +256,7 @@ def run_reference(args, rank, world):
     params = sub.shape[0] * sub.shape[1]
     step = statistics.mean(times)
     value = params / step / 1e9
-    line = {"impl": "reference", "metric": "transposable N:M mask Gparams/s (oracle, host cores)",
+    line = {"impl": "reference", "metric": METRIC,
             "value": value, "unit": "Gparams/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": step * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
@@ -317,7 +318,7 @@ def run_stack(args, rank, world):
     clocks = sampler.stop()
     tsl.tsenor_error_count()
     line = {
-        "metric": "transposable N:M mask Gparams/s at 1 B200 (% of roofline); mean gap to exact opt",
+        "metric": METRIC,
         "value": aggregate_gparams(params, world, ms_max), "unit": "Gparams/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
@@ -427,7 +428,7 @@ def run_warm(args, rank, world):
     ops = params * mean_iters * (1.0 + 2.0 / w.M)
     peak = mufu_peak_tops(SM_MAX_MHZ_FALLBACK)
     line = {
-        "metric": "transposable N:M mask Gparams/s at 1 B200 (% of roofline); mean gap to exact opt",
+        "metric": METRIC,
         "value": aggregate_gparams(params, world, ms_max), "unit": "Gparams/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
@@ -585,7 +586,7 @@ def main(argv=None):
     achieved = params * ops_per_param / (kernel_ms / 1e3) / 1e12
     traffic = profiled_traffic(kernel_key)
     line = {
-        "metric": "transposable N:M mask Gparams/s at 1 B200 (% of roofline); mean gap to exact opt",
+        "metric": METRIC,
         "value": value, "unit": "Gparams/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": mean_ms_max, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
