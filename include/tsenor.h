@@ -213,6 +213,28 @@ tsenor_status tsenor_plan_warm(const void* W, tsenor_dtype dtype, int64_t rows, 
 tsenor_status tsenor_mask_scores(const float* scores, int64_t rows, int64_t cols, int N, int M, float tau,
                                  int iters, int sweeps, uint32_t* mask_out, tsenor_stream_t stream);
 
+/*
+ * tsenor_mask for W and the mask in HOST memory, with the transfers
+ * overlapped with the solve: W is cut into row chunks (multiples of M rows);
+ * chunk k+1 is copied to the device while chunk k is solved, and each
+ * chunk's mask is copied back as soon as it is ready.  Results are those of
+ * tsenor_mask on the whole matrix (blocks are independent).
+ *   W_host:    rows x cols, row-major, host memory; page-locked memory
+ *              (cudaHostAlloc / cudaHostRegister) lets the copies overlap,
+ *              pageable memory works but serialises them.
+ *   mask_host: rows x words_per_row uint32, host memory (page-locked for
+ *              overlap); written completely.
+ *   stream:    every copy and kernel is ordered after the work already on
+ *              `stream`, and `stream` waits for all of them before its later
+ *              work (the library uses two internal streams in between).  The
+ *              host buffers must stay valid until then.
+ * Uses stream-ordered device workspaces for two W chunks and two mask chunks
+ * (cudaMallocAsync / cudaFreeAsync).  Errors as tsenor_mask; TSENOR_ERR_ARG
+ * also for a null host pointer.  The review has no counterpart of this call.
+ */
+tsenor_status tsenor_mask_host(const void* W_host, tsenor_dtype dtype, int64_t rows, int64_t cols, int N, int M,
+                               float tau, int iters, int sweeps, uint32_t* mask_host, tsenor_stream_t stream);
+
 /* Static description of a status code. */
 const char* tsenor_status_string(int status);
 

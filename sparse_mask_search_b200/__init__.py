@@ -18,7 +18,7 @@ STATUS = {0: "TSENOR_OK", -1: "TSENOR_ERR_ARG", -2: "TSENOR_ERR_SHAPE", -3: "TSE
 NOALLOC_MAX_PARAMS = 16 * 1024 * 1024
 EXPORTS = ("tsenor_mask", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
            "tsenor_status_string", "tsenor_last_error", "tsenor_mask_noalloc", "tsenor_mask_safeguard",
-           "tsenor_mask_padded", "tsenor_mask_warm", "tsenor_plan_warm", "tsenor_mask_scores")
+           "tsenor_mask_padded", "tsenor_mask_warm", "tsenor_plan_warm", "tsenor_mask_scores", "tsenor_mask_host")
 
 _lib = None
 
@@ -44,6 +44,7 @@ def lib() -> C.CDLL:
         L.tsenor_mask_padded.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p]
         L.tsenor_mask_safeguard.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p, p, p]
         L.tsenor_mask_scores.argtypes = [p, i64, i64, i32, i32, f32, i32, i32, p, p]
+        L.tsenor_mask_host.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, p, p]
         L.tsenor_mask_warm.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, i32, f32, i32, p, p, p, p]
         L.tsenor_plan_warm.argtypes = [p, i32, i64, i64, i32, i32, f32, i32, f32, i32, p, p, p, p]
         L.tsenor_round.argtypes = [p, p, i32, i64, i64, i32, i32, i32, p, p]
@@ -154,6 +155,27 @@ def tsenor_mask_scores(scores, N: int, M: int, tau: float, iters: int, sweeps: i
         out = torch.empty((rows, words_per_row(cols)), dtype=torch.int32, device=scores.device)
     _check(lib().tsenor_mask_scores(scores.data_ptr(), rows, cols, N, M, float(tau), iters, sweeps, out.data_ptr(),
                                     _stream_handle(stream)))
+    return out
+
+
+def tsenor_mask_host(W_host, N: int, M: int, tau: float, iters: int, sweeps: int, out=None, stream=None):
+    """tsenor_mask of a HOST matrix into a HOST mask, the copies overlapped with the solve.
+
+    W_host: contiguous 2-D CPU tensor (bfloat16 or float32), ideally pinned.
+    Returns the (rows, ceil(cols/32)) int32 mask on the host (pinned when
+    allocated here).  The result is complete once ``stream`` (default: the
+    current CUDA stream) reaches this point, e.g. after its synchronize().
+    """
+    import torch
+    if W_host.is_cuda or W_host.dim() != 2 or not W_host.is_contiguous():
+        raise ValueError("W_host must be a contiguous 2-D CPU tensor")
+    rows, cols = W_host.shape
+    if out is None:
+        out = torch.empty((rows, words_per_row(cols)), dtype=torch.int32, pin_memory=True)
+    elif out.is_cuda or not out.is_contiguous() or out.numel() < rows * words_per_row(cols):
+        raise ValueError("out must be a contiguous CPU int32 tensor of (rows, ceil(cols/32))")
+    _check(lib().tsenor_mask_host(W_host.data_ptr(), _dtype_code(W_host), rows, cols, N, M, float(tau), iters,
+                                  sweeps, out.data_ptr(), _stream_handle(stream)))
     return out
 
 
@@ -273,6 +295,6 @@ def tsenor_error_count(stream=None) -> int:
     return int(n.value)
 
 
-__all__ = ["tsenor_mask", "tsenor_mask_scores", "tsenor_mask_noalloc", "tsenor_mask_safeguard", "tsenor_mask_padded", "tsenor_mask_warm",
+__all__ = ["tsenor_mask", "tsenor_mask_host", "tsenor_mask_scores", "tsenor_mask_noalloc", "tsenor_mask_safeguard", "tsenor_mask_padded", "tsenor_mask_warm",
            "tsenor_plan", "tsenor_plan_warm", "tsenor_round", "tsenor_objective", "tsenor_error_count",
            "TsenorError", "lib", "words_per_row", "EXPORTS", "LIB_PATH"]

@@ -343,6 +343,118 @@ extern "C" tsenor_status tsenor_plan_warm(const void* W, tsenor_dtype dtype, int
     return e == cudaSuccess ? TSENOR_OK : cuda_fail(e, "tsenor_plan_warm launch");
 }
 
+// ---------------------------------------------------------------------------
+// tsenor_mask_host: row chunks of a host matrix pipelined through two device
+// slots.  Copies run on an internal stream X, solves alternate between the
+// caller's stream and a second internal stream (so that one chunk's tail
+// overlaps the next chunk's head).  X first uploads chunks 0 and 1; then per
+// chunk k, slot s = k % 2:
+//   compute stream: wait h2d[k]; tsenor_mask on dW[s] -> dmask[s]; event comp[k]
+//   X: wait comp[k]; copy dmask[s] -> host mask chunk k; upload chunk k+2
+//      into dW[s] (free: chunk k's solve is done); event h2d[k+2]
+// so each upload overlaps the solve of the chunk before it.  The caller's
+// stream then waits for X's last copy.
+namespace {
+constexpr int kHostMaxChunks = 64;
+
+struct HostPipe {
+    cudaStream_t x = nullptr, c2 = nullptr;
+    cudaEvent_t ev[2 * kHostMaxChunks + 2] = {};
+    int nev = 0;
+    void* dW[2] = {nullptr, nullptr};
+    uint32_t* dm[2] = {nullptr, nullptr};
+    cudaEvent_t event() {
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+        ev[nev++] = e;
+        return e;
+    }
+    void release(cudaStream_t st) {
+        for (int s = 0; s < 2; ++s) {
+            if (dW[s]) cudaFreeAsync(dW[s], st);
+            if (dm[s]) cudaFreeAsync(dm[s], st);
+        }
+        for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
+        if (x) cudaStreamDestroy(x);
+        if (c2) cudaStreamDestroy(c2);
+    }
+};
+}  // namespace
+
+extern "C" tsenor_status tsenor_mask_host(const void* W_host, tsenor_dtype dtype, int64_t rows, int64_t cols, int N,
+                                          int M, float tau, int iters, int sweeps, uint32_t* mask_host,
+                                          tsenor_stream_t stream) {
+    if (M != 4 && M != 8 && M != 16 && M != 32 && M != 64) return TSENOR_ERR_UNSUPPORTED_M;
+    if (dtype != TSENOR_F32 && dtype != TSENOR_BF16) return TSENOR_ERR_ARG;
+    if (N < 1 || N > M || !solver_params_ok(tau, iters) || sweeps < 0) return TSENOR_ERR_ARG;
+    if (rows < 0 || cols < 0 || rows % M || cols % M) return TSENOR_ERR_SHAPE;
+    if (rows > (int64_t(1) << 31) || cols > (int64_t(1) << 31)) return TSENOR_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return TSENOR_OK;
+    if (!W_host || !mask_host) return TSENOR_ERR_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t es = dtype == TSENOR_BF16 ? 2 : 4;
+    const int64_t wpr = (cols + 31) / 32;
+    // one chunk per ~8 MB of W, between 1 and 8 chunks, each a multiple of M rows
+    const int64_t bytes = rows * cols * int64_t(es);
+    int64_t want = bytes / (int64_t(8) << 20);
+    want = want < 1 ? 1 : (want > 8 ? 8 : want);
+    int64_t chunk = ((rows + want - 1) / want + M - 1) / M * M;
+    const int64_t nchunks = (rows + chunk - 1) / chunk;
+
+    HostPipe p;
+    cudaError_t e = cudaStreamCreateWithFlags(&p.x, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p.c2, cudaStreamNonBlocking);
+    for (int s = 0; s < 2 && e == cudaSuccess; ++s) {
+        e = cudaMallocAsync(&p.dW[s], size_t(chunk) * size_t(cols) * es, st);
+        if (e == cudaSuccess)
+            e = cudaMallocAsync(reinterpret_cast<void**>(&p.dm[s]), size_t(chunk) * size_t(wpr) * 4, st);
+    }
+    cudaEvent_t start = e == cudaSuccess ? p.event() : nullptr;
+    if (e == cudaSuccess && !start) e = cudaErrorMemoryAllocation;
+    // everything below is ordered after the caller's earlier work and the allocations
+    if (e == cudaSuccess) e = cudaEventRecord(start, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(p.x, start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(p.c2, start, 0);
+    tsenor_status s = TSENOR_OK;
+    cudaEvent_t h2d[kHostMaxChunks] = {};
+    auto rows_of = [&](int64_t k) { return rows - k * chunk < chunk ? rows - k * chunk : chunk; };
+    auto upload = [&](int64_t k) -> cudaError_t {        // on X: W chunk k into slot k % 2
+        h2d[k] = p.event();
+        if (!h2d[k]) return cudaErrorMemoryAllocation;
+        cudaError_t r = cudaMemcpyAsync(p.dW[k % 2],
+                                        static_cast<const char*>(W_host) + size_t(k * chunk) * size_t(cols) * es,
+                                        size_t(rows_of(k)) * size_t(cols) * es, cudaMemcpyHostToDevice, p.x);
+        return r == cudaSuccess ? cudaEventRecord(h2d[k], p.x) : r;
+    };
+    for (int64_t k = 0; k < 2 && k < nchunks && e == cudaSuccess; ++k) e = upload(k);
+    for (int64_t k = 0; k < nchunks && e == cudaSuccess && s == TSENOR_OK; ++k) {
+        const int slot = int(k % 2);
+        const int64_t r0 = k * chunk, nr = rows_of(k);
+        cudaStream_t cs = slot == 0 ? st : p.c2;
+        cudaEvent_t comp = p.event();
+        if (!comp) { e = cudaErrorMemoryAllocation; break; }
+        e = cudaStreamWaitEvent(cs, h2d[k], 0);
+        if (e != cudaSuccess) break;
+        s = tsenor_mask(p.dW[slot], dtype, nr, cols, N, M, tau, iters, sweeps, p.dm[slot], (tsenor_stream_t)cs);
+        if (s != TSENOR_OK) break;
+        e = cudaEventRecord(comp, cs);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(p.x, comp, 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(mask_host + size_t(r0) * size_t(wpr), p.dm[slot], size_t(nr) * size_t(wpr) * 4,
+                                cudaMemcpyDeviceToHost, p.x);
+        if (e == cudaSuccess && k + 2 < nchunks) e = upload(k + 2);
+    }
+    // the caller's stream waits for the last copy (and with it every chunk)
+    cudaEvent_t done = p.event();
+    cudaError_t e2 = done ? cudaEventRecord(done, p.x) : cudaErrorMemoryAllocation;
+    if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, done, 0);
+    p.release(st);
+    if (s != TSENOR_OK) return s;
+    if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask_host");
+    if (e2 != cudaSuccess) return cuda_fail(e2, "tsenor_mask_host join");
+    return TSENOR_OK;
+}
+
 extern "C" tsenor_status tsenor_mask_safeguard(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
                                                int N, int M, float tau, int iters, int sweeps,
                                                const uint32_t* prev_mask, uint32_t* mask_out,

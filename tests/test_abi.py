@@ -102,6 +102,15 @@ def test_scores_entry_point_validates():
     assert L.tsenor_mask_scores(0, 0, 64, 2, 4, 10.0, 5, 1, 0, None) == 0                   # empty
 
 
+def test_host_entry_point_validates():
+    L = tsl.lib()
+    assert L.tsenor_mask_host(None, 1, 64, 64, 2, 4, 10.0, 5, 1, 1 << 12, None) == -1     # no W
+    assert L.tsenor_mask_host(1 << 12, 1, 64, 64, 2, 4, 10.0, 5, 1, None, None) == -1     # no mask
+    assert L.tsenor_mask_host(1 << 12, 1, 64, 62, 2, 4, 10.0, 5, 1, 1 << 12, None) == -2
+    assert L.tsenor_mask_host(1 << 12, 1, 64, 64, 2, 6, 10.0, 5, 1, 1 << 12, None) == -3
+    assert L.tsenor_mask_host(None, 1, 0, 64, 2, 4, 10.0, 5, 1, None, None) == 0          # empty
+
+
 def test_warm_empty_calls_do_nothing():
     L = tsl.lib()
     assert _warm(L, rows=0, W=0, out=0, pot=0, used=0) == 0

@@ -97,3 +97,24 @@ def test_padded_shapes(rows, cols, M, N, dtype):
         for c0 in range(0, cols, M):
             blk = bits[r0:r0 + M, c0:c0 + M]
             assert (blk.sum(axis=1) <= N).all() and (blk.sum(axis=0) <= N).all()
+
+
+@pytest.mark.parametrize("rows,cols,M,N,dtype", [(4096, 1024, 32, 16, "bf16"), (1000 // 8 * 8, 96, 8, 4, "f32"),
+                                                 (64, 64, 16, 8, "bf16"), (8 * 64, 128, 64, 32, "bf16"),
+                                                 (36, 40, 4, 2, "f32"),
+                                                 # 17 MB and 32 MB of W: two and four chunks, the last one shorter
+                                                 (4192, 2048, 32, 16, "bf16"), (4096, 2048, 8, 4, "f32")])
+def test_host_pipeline_matches_device_call(rows, cols, M, N, dtype):
+    """tsenor_mask_host (row chunks of ~8 MB pipelined through two device slots) gives tsenor_mask's mask."""
+    stor, W = synth.make_matrix(rows, cols, dtype, "t3_outlier_cols", 0.02, seed=rows + M)
+    Wd = to_device(stor, dtype)
+    ref = tsl.tsenor_mask(Wd, N, M, 20.0, 120, 4).cpu()
+    Wh = Wd.cpu().pin_memory()
+    side = torch.cuda.Stream()
+    out = tsl.tsenor_mask_host(Wh, N, M, 20.0, 120, 4, stream=side)
+    side.synchronize()
+    assert torch.equal(out, ref)
+    # pageable buffers work too
+    out2 = tsl.tsenor_mask_host(Wd.cpu(), N, M, 20.0, 120, 4, out=torch.zeros_like(ref))
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(out2, ref)
