@@ -72,9 +72,8 @@ typedef enum {
  * repair, local search, bit packing).
  *   mask_out: rows x words_per_row uint32, written completely.
  *   sweeps:   local-search sweeps L; one sweep visits every anchor row once.
- * M = 16, 32, 64: one fused kernel, no workspace.  M = 4, 8: a plan kernel
- * and a rounding kernel with a stream-ordered workspace of rows*cols floats
- * between them (cudaMallocAsync / cudaFreeAsync on `stream`).
+ * One fused kernel per call (every M), no workspace: the plan never leaves
+ * the chip.
  */
 tsenor_status tsenor_mask(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols,
                           int N, int M, float tau, int iters, int sweeps,

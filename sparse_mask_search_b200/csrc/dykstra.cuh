@@ -52,16 +52,12 @@ __device__ __forceinline__ float plan_value(float y) { return y >= 0.f ? 1.f : e
 // the exponentials of one row live only until its column contributions are
 // added, so no cross-thread traffic is needed at all.
 // ---------------------------------------------------------------------------
+// Dykstra for block b (rows r0.., columns c0..) by one thread.  On return y
+// holds the final state; returns whether the block's W is finite.
 template <int M, typename T, bool EXT = false>
-__global__ void __launch_bounds__(128)
-dykstra_thread_kernel(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks,
-                      int N, float tau, int iters, float* __restrict__ plan, DykstraExt ext = {}) {
-    const int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (b >= n_blocks) return;
-    const int64_t nbc = cols / M;
-    const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
-
-    float y[M][M];
+__device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* __restrict__ W, int64_t cols,
+                                                     int64_t b, int64_t r0, int64_t c0, int N, float tau,
+                                                     int iters, const DykstraExt& ext, float (&y)[M][M]) {
 #pragma unroll
     for (int i = 0; i < M; ++i) {
         const typename T::storage* src = W + (r0 + i) * cols + c0;
@@ -177,6 +173,19 @@ dykstra_thread_kernel(const typename T::storage* __restrict__ W, int64_t cols, i
         }
         if (ext.iters_used) ext.iters_used[b] = finite ? used : 0;
     }
+    return finite;
+}
+
+template <int M, typename T, bool EXT = false>
+__global__ void __launch_bounds__(128)
+dykstra_thread_kernel(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks,
+                      int N, float tau, int iters, float* __restrict__ plan, DykstraExt ext = {}) {
+    const int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (b >= n_blocks) return;
+    const int64_t nbc = cols / M;
+    const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
+    float y[M][M];
+    const bool finite = dykstra_thread_solve<M, T, EXT>(W, cols, b, r0, c0, N, tau, iters, ext, y);
 #pragma unroll
     for (int i = 0; i < M; ++i) {
         float s[M];

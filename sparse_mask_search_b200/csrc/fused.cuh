@@ -14,17 +14,21 @@
 #include <type_traits>
 
 #include "dykstra.cuh"
+#include "round_group.cuh"
 #include "round_warp.cuh"
 
 namespace tsenor {
 
-// bf16: registers capped for 5 CTAs (20 warps) per SM (5.00 ms against 5.03 ms
-// uncapped on the 4096x11008 16:32 workload); the fp32 key needs more.
+// bf16: registers capped at 80 (the bound for 6 CTAs per SM; shared memory
+// still admits 5, so only the generated code changes): 4.98 ms against 5.01 ms
+// with the 96-register cap of 5 CTAs and 5.03 ms uncapped on the 4096x11008
+// 16:32 workload, in two runs each.  The fp32 key needs more registers; the
+// EXT instance keeps the 96-register cap.
 // The tile is read with 16-byte loads here, not staged by TMA: on the same
 // workload the TMA-staged variant of this kernel timed 5.16 ms against
 // 5.01 ms (the plan kernel of the same M gained 0.7% from TMA staging).
 template <typename T, bool EXT = false>
-__global__ void __launch_bounds__(128, std::is_same<T, BF16>::value ? 5 : 4)
+__global__ void __launch_bounds__(128, std::is_same<T, BF16>::value ? (EXT ? 5 : 6) : 4)
 fused_kernel32(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
                int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr, DykstraExt ext = {}) {
     constexpr int M = 32;
@@ -132,6 +136,80 @@ constexpr size_t fused16_smem() {
 }
 static_assert((sizeof(float) * 16 * (16 * 17 + 16 * 16) + sizeof(RoundShared<16>) * 4 + sizeof(int) * 16) % 8 == 0,
               "barrier alignment");
+
+// M = 4, 8: a CTA of 64 threads solves 64 blocks, one per thread (the whole
+// block in registers, as dykstra_thread_kernel), stages the plans in shared
+// memory, then groups of M lanes round them (round_group.cuh), each group
+// several blocks in turn; |W| for the keys is read again (from L2).
+template <int M>
+struct FusedSmallCfg {
+    static constexpr int THREADS = 64;                         // = blocks per CTA
+    static constexpr int SS = M * M + 4;                       // plan row stride (floats; conflict-free stores)
+    static constexpr int NG = THREADS / M;                     // groups per CTA
+    static constexpr size_t plan_bytes = sizeof(float) * THREADS * SS;
+    static constexpr size_t group_off = plan_bytes;
+    static constexpr size_t flags_off = group_off + sizeof(RoundGroupSmem<M>) * NG;
+    static constexpr size_t bytes = flags_off + sizeof(int) * THREADS;
+};
+
+template <int M, typename T, bool EXT = false>
+__global__ void __launch_bounds__(64)
+fused_kernel_small(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
+                   int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr, DykstraExt ext = {}) {
+    using Cfg = FusedSmallCfg<M>;
+    using Key = typename KeyOf<T>::type;
+    constexpr int AS = M + 1;
+    extern __shared__ __align__(16) unsigned char fused_small_raw[];
+    float* plans = reinterpret_cast<float*>(fused_small_raw);
+    RoundGroupSmem<M>* groups = reinterpret_cast<RoundGroupSmem<M>*>(fused_small_raw + Cfg::group_off);
+    int* flags = reinterpret_cast<int*>(fused_small_raw + Cfg::flags_off);
+    const int t = threadIdx.x;
+    const int64_t nbc = cols / M;
+    {
+        const int64_t b = int64_t(blockIdx.x) * Cfg::THREADS + t;
+        if (b < n_blocks) {
+            const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
+            float y[M][M];
+            const bool finite = dykstra_thread_solve<M, T, EXT>(W, cols, b, r0, c0, N, tau, iters, ext, y);
+            float* dst = plans + t * Cfg::SS;
+#pragma unroll
+            for (int i = 0; i < M; ++i)
+#pragma unroll
+                for (int v = 0; v < M / 4; ++v)
+                    reinterpret_cast<float4*>(dst + i * M)[v] =
+                        make_float4(plan_value(y[i][4 * v]), plan_value(y[i][4 * v + 1]),
+                                    plan_value(y[i][4 * v + 2]), plan_value(y[i][4 * v + 3]));
+            flags[t] = finite;
+        }
+    }
+    __syncthreads();
+
+    const int lane = t & 31, gl = lane % M, g = t / M;
+    const unsigned gmask = ((1u << M) - 1u) << (lane - gl);
+    RoundGroupSmem<M>& sm = groups[g];
+    const RoundView<M> sh = sm.sh.view();
+    for (int s = g; s < Cfg::THREADS; s += Cfg::NG) {
+        const int64_t b = int64_t(blockIdx.x) * Cfg::THREADS + s;
+        if (b >= n_blocks) break;                             // uniform per group
+        const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
+        const float* src = plans + s * Cfg::SS;
+        Key key[M];
+#pragma unroll
+        for (int r = 0; r < M; ++r) {
+            const int e = r * M + gl;                         // row r, column gl
+            const float a = T::load1(W + (r0 + r) * cols + c0 + gl);
+            sm.a[r * AS + gl] = a;
+            key[r] = Key::make(src[e], a, e);
+        }
+        __syncwarp(gmask);
+        bool ok = flags[s] != 0;
+        if (ok) ok = round_block_group<M, Key>(key, sm.a, sh, N, sweeps, lane, gl, gmask);
+        if (!ok && gl == 0) atomicAdd(&g_block_failures, 1ull);
+        __syncwarp(gmask);
+        write_group_row<M>(mask, wpr, r0, c0, ok ? static_cast<unsigned>(sh.rowbits[gl]) : 0u, gl);
+        __syncwarp(gmask);                                    // the group's arrays are reused by its next block
+    }
+}
 
 // M = 64: one CTA of 4 warps per block; Round64Smem's colbuf serves the
 // Dykstra phase's cross-warp column sums.

@@ -218,6 +218,38 @@ __device__ void group_local_search(const float* a, const RoundView<M>& sh, int s
     }
 }
 
+// Steps 1-4 for one block by its group: `key` holds lane gl's keys (entry
+// r*M + gl in register r), `a` the block's |W| (row stride M+1, shared
+// memory).  Returns false when the block could not be made feasible; the
+// row bitmasks are in sh.rowbits.
+template <int M, typename Key>
+__device__ __forceinline__ bool round_block_group(Key (&key)[M], const float* a, const RoundView<M>& sh, int N,
+                                                  int sweeps, int lane, int gl, unsigned gmask) {
+    group_bitonic_sort<M, M>(key, gl, gmask);
+#pragma unroll
+    for (int r = 0; r < M; ++r) sh.order[gl * M + r] = static_cast<uint16_t>(key[r].index());
+    __syncwarp(gmask);
+    if (!group_greedy_and_repair<M>(a, sh, N, lane, gl, gmask)) return false;
+    if (sweeps > 0) {
+        __syncwarp(gmask);
+        group_local_search<M>(a, sh, sweeps, gl, gmask);
+    }
+    return true;
+}
+
+// Row gl of a block's mask: a byte (M = 8) or a nibble OR-ed into a zeroed
+// mask (M = 4).
+template <int M>
+__device__ __forceinline__ void write_group_row(uint32_t* mask, int64_t wpr, int64_t r0, int64_t c0, unsigned bits,
+                                                int gl) {
+    uint32_t* row = mask + (r0 + gl) * wpr;
+    if constexpr (M == 8) {
+        reinterpret_cast<uint8_t*>(row)[c0 / 8] = static_cast<uint8_t>(bits);
+    } else {
+        if (bits) atomicOr(&row[c0 / 32], bits << (c0 % 32));
+    }
+}
+
 // Rounding of a given plan, M lanes per block (M = 4, 8).  Entry e = r*M + gl
 // of the block goes to lane gl's register r: register r holds block row r,
 // so a group reads whole block rows and the groups of a warp read
@@ -256,28 +288,12 @@ round_group_kernel(const float* __restrict__ plan, const typename T::storage* __
         key[r] = Key::make(s, a, e);
     }
     ok = __all_sync(gmask, ok);
+    __syncwarp(gmask);
     const RoundView<M> sh = sm.sh.view();
-    if (ok) {
-        group_bitonic_sort<R, G>(key, gl, gmask);
-#pragma unroll
-        for (int r = 0; r < R; ++r) sh.order[gl * R + r] = static_cast<uint16_t>(key[r].index());
-        __syncwarp(gmask);
-        ok = group_greedy_and_repair<M>(sm.a, sh, N, lane, gl, gmask);
-        if (ok && sweeps > 0) {
-            __syncwarp(gmask);
-            group_local_search<M>(sm.a, sh, sweeps, gl, gmask);
-        }
-    }
+    if (ok) ok = round_block_group<M, Key>(key, sm.a, sh, N, sweeps, lane, gl, gmask);
     if (!ok && gl == 0) atomicAdd(&g_block_failures, 1ull);
     __syncwarp(gmask);
-    // row gl of the block: a byte (M = 8) or a nibble OR-ed into a zeroed mask (M = 4)
-    const unsigned bits = ok ? static_cast<unsigned>(sh.rowbits[gl]) : 0u;
-    uint32_t* row = mask + (r0 + gl) * wpr;
-    if constexpr (M == 8) {
-        reinterpret_cast<uint8_t*>(row)[c0 / 8] = static_cast<uint8_t>(bits);
-    } else {
-        if (bits) atomicOr(&row[c0 / 32], bits << (c0 % 32));
-    }
+    write_group_row<M>(mask, wpr, r0, c0, ok ? static_cast<unsigned>(sh.rowbits[gl]) : 0u, gl);
 }
 
 template <int M>

@@ -135,7 +135,20 @@ cudaError_t launch_fused(const void* W, int64_t rows, int64_t cols, int N, float
     const int64_t nb = (rows / M) * (cols / M);
     const int64_t wpr = (cols + 31) / 32;
     cudaError_t e = cudaSuccess;
-    if constexpr (M == 32) {
+    if constexpr (M <= 8) {
+        if (M == 4 || cols % 32) {
+            // sub-word rows: zero first so padding bits are 0 (and M = 4 can OR)
+            e = cudaMemsetAsync(mask, 0, size_t(rows) * size_t(wpr) * 4, st);
+            if (e != cudaSuccess) return e;
+        }
+        constexpr size_t smem = FusedSmallCfg<M>::bytes;
+        e = cudaFuncSetAttribute(fused_kernel_small<M, T, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(smem));
+        if (e != cudaSuccess) return e;
+        constexpr int64_t bpc = FusedSmallCfg<M>::THREADS;
+        fused_kernel_small<M, T, EXT><<<dim3(unsigned((nb + bpc - 1) / bpc)), FusedSmallCfg<M>::THREADS, smem, st>>>(
+            static_cast<const typename T::storage*>(W), cols, nb, N, tau, iters, sweeps, mask, wpr, ext);
+    } else if constexpr (M == 32) {
         const auto* w = static_cast<const typename T::storage*>(W);
         constexpr size_t smem = fused32_smem();
         e = cudaFuncSetAttribute(fused_kernel32<T, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
@@ -173,6 +186,8 @@ template <typename T, bool EXT>
 cudaError_t dispatch_fused_m(int M, const void* W, int64_t rows, int64_t cols, int N, float tau, int iters,
                              int sweeps, uint32_t* mask, cudaStream_t st, const DykstraExt& ext) {
     switch (M) {
+        case 4: return launch_fused<4, T, EXT>(W, rows, cols, N, tau, iters, sweeps, mask, st, ext);
+        case 8: return launch_fused<8, T, EXT>(W, rows, cols, N, tau, iters, sweeps, mask, st, ext);
         case 16: return launch_fused<16, T, EXT>(W, rows, cols, N, tau, iters, sweeps, mask, st, ext);
         case 32: return launch_fused<32, T, EXT>(W, rows, cols, N, tau, iters, sweeps, mask, st, ext);
         default: return launch_fused<64, T, EXT>(W, rows, cols, N, tau, iters, sweeps, mask, st, ext);
@@ -279,20 +294,9 @@ extern "C" tsenor_status tsenor_mask(const void* W, tsenor_dtype dtype, int64_t 
     if (rows == 0 || cols == 0) return TSENOR_OK;
     if (!mask_out || !aligned(mask_out, 8)) return TSENOR_ERR_ARG;
     cudaStream_t st = (cudaStream_t)stream;
-    if (M >= 16) {
-        cudaError_t e = dtype == TSENOR_BF16 ? dispatch_fused<BF16>(M, W, rows, cols, N, tau, iters, sweeps, mask_out, st)
-                                             : dispatch_fused<F32>(M, W, rows, cols, N, tau, iters, sweeps, mask_out, st);
-        return e == cudaSuccess ? TSENOR_OK : cuda_fail(e, "tsenor_mask launch");
-    }
-    float* plan = nullptr;
-    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&plan), size_t(rows) * size_t(cols) * sizeof(float), st);
-    if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask workspace");
-    e = run_plan(dtype, M, W, rows, cols, N, tau, iters, plan, st);
-    if (e == cudaSuccess) e = run_round(dtype, M, plan, W, rows, cols, N, sweeps, mask_out, st);
-    cudaError_t e2 = cudaFreeAsync(plan, st);
-    if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask launch");
-    if (e2 != cudaSuccess) return cuda_fail(e2, "tsenor_mask workspace free");
-    return TSENOR_OK;
+    cudaError_t e = dtype == TSENOR_BF16 ? dispatch_fused<BF16>(M, W, rows, cols, N, tau, iters, sweeps, mask_out, st)
+                                         : dispatch_fused<F32>(M, W, rows, cols, N, tau, iters, sweeps, mask_out, st);
+    return e == cudaSuccess ? TSENOR_OK : cuda_fail(e, "tsenor_mask launch");
 }
 
 extern "C" tsenor_status tsenor_mask_scores(const float* scores, int64_t rows, int64_t cols, int N, int M, float tau,
@@ -312,21 +316,10 @@ extern "C" tsenor_status tsenor_mask_warm(const void* W, tsenor_dtype dtype, int
     if (!mask_out || !aligned(mask_out, 8)) return TSENOR_ERR_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     const DykstraExt ext{potentials, iters_used, tol * kLog2e, warm != 0};
-    if (M >= 16) {
-        cudaError_t e = dtype == TSENOR_BF16
-                            ? dispatch_fused<BF16>(M, W, rows, cols, N, tau, iters, sweeps, mask_out, st, &ext)
-                            : dispatch_fused<F32>(M, W, rows, cols, N, tau, iters, sweeps, mask_out, st, &ext);
-        return e == cudaSuccess ? TSENOR_OK : cuda_fail(e, "tsenor_mask_warm launch");
-    }
-    float* plan = nullptr;
-    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&plan), size_t(rows) * size_t(cols) * sizeof(float), st);
-    if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask_warm workspace");
-    e = run_plan(dtype, M, W, rows, cols, N, tau, iters, plan, st, &ext);
-    if (e == cudaSuccess) e = run_round(dtype, M, plan, W, rows, cols, N, sweeps, mask_out, st);
-    cudaError_t e2 = cudaFreeAsync(plan, st);
-    if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask_warm launch");
-    if (e2 != cudaSuccess) return cuda_fail(e2, "tsenor_mask_warm workspace free");
-    return TSENOR_OK;
+    cudaError_t e = dtype == TSENOR_BF16
+                        ? dispatch_fused<BF16>(M, W, rows, cols, N, tau, iters, sweeps, mask_out, st, &ext)
+                        : dispatch_fused<F32>(M, W, rows, cols, N, tau, iters, sweeps, mask_out, st, &ext);
+    return e == cudaSuccess ? TSENOR_OK : cuda_fail(e, "tsenor_mask_warm launch");
 }
 
 extern "C" tsenor_status tsenor_plan_warm(const void* W, tsenor_dtype dtype, int64_t rows, int64_t cols, int N,
