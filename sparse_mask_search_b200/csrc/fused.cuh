@@ -139,8 +139,9 @@ static_assert((sizeof(float) * 16 * (16 * 17 + 16 * 16) + sizeof(RoundShared<16>
 
 // M = 4, 8: a CTA of 64 threads solves 64 blocks, one per thread (the whole
 // block in registers, as dykstra_thread_kernel), stages the plans in shared
-// memory, then groups of M lanes round them (round_group.cuh), each group
-// several blocks in turn; |W| for the keys is read again (from L2).
+// memory, then groups of M lanes of each warp round that warp's 32 blocks
+// (round_group.cuh), each group several in turn; |W| for the keys is read
+// again (from L2).
 template <int M>
 struct FusedSmallCfg {
     static constexpr int THREADS = 64;                         // = blocks per CTA
@@ -182,13 +183,16 @@ fused_kernel_small(const typename T::storage* __restrict__ W, int64_t cols, int6
             flags[t] = finite;
         }
     }
-    __syncthreads();
+    // each warp rounds the 32 blocks its own lanes solved: no CTA-wide barrier,
+    // so warps drift apart and one warp's rounding overlaps another's solve
+    __syncwarp();
 
     const int lane = t & 31, gl = lane % M, g = t / M;
     const unsigned gmask = ((1u << M) - 1u) << (lane - gl);
     RoundGroupSmem<M>& sm = groups[g];
     const RoundView<M> sh = sm.sh.view();
-    for (int s = g; s < Cfg::THREADS; s += Cfg::NG) {
+    const int wbase = t - lane;                               // first block slot of this warp
+    for (int s = wbase + lane / M; s < wbase + 32; s += 32 / M) {
         const int64_t b = int64_t(blockIdx.x) * Cfg::THREADS + s;
         if (b >= n_blocks) break;                             // uniform per group
         const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;

@@ -259,13 +259,22 @@ __device__ bool greedy_and_repair(const float* a, const RoundView<M>& sh, int N,
     __syncwarp();
     const int target = N * M;
     int taken = 0;
+    const unsigned lt = (1u << lane) - 1u;
+    // the next chunk's entries and row/column groups do not depend on this
+    // chunk's decisions: they are fetched one chunk ahead
+    int e_next = sh.order[lane];
+    unsigned mr_next = __match_any_sync(kFullMask, e_next < E ? e_next / M : 4096 + lane);
+    unsigned mc_next = __match_any_sync(kFullMask, e_next < E ? e_next % M : 8192 + lane);
     for (int base = 0; base < EP && taken < target; base += 32) {
-        const int e = sh.order[base + lane];
+        const int e = e_next;
+        const unsigned mr = mr_next, mc = mc_next;
+        if (base + 32 < EP) {
+            e_next = sh.order[base + 32 + lane];
+            mr_next = __match_any_sync(kFullMask, e_next < E ? e_next / M : 4096 + lane);
+            mc_next = __match_any_sync(kFullMask, e_next < E ? e_next % M : 8192 + lane);
+        }
         const bool valid = e < E;
         const int i = valid ? e / M : 0, j = valid ? e % M : 0;
-        const unsigned mr = __match_any_sync(kFullMask, valid ? i : 4096 + lane);
-        const unsigned mc = __match_any_sync(kFullMask, valid ? j : 8192 + lane);
-        const unsigned lt = (1u << lane) - 1u;
         const int r0c = valid ? sh.rc[i] : N, c0c = valid ? sh.cc[j] : N;
         unsigned acc = 0u;
         unsigned und = __ballot_sync(kFullMask, valid && r0c < N && c0c < N);
