@@ -520,12 +520,13 @@ __device__ bool round_block_warp(Key (&key)[WarpRound<M>::R], const float* a, co
     return true;
 }
 
-// Row bitmasks of one block into the packed mask (M >= 8: whole bytes,
-// halves or words; M = 4: OR into a zeroed mask, two blocks share a byte).
+// Row bitmasks of one block into the packed mask as whole words or halves
+// (M = 16, 32, 64; the small-block kernels write their rows themselves).
 template <int M>
 __device__ __forceinline__ void write_mask_rows(uint32_t* mask, int64_t wpr, int64_t r0, int64_t c0,
                                                 const typename WarpRound<M>::Bits* rowbits, bool ok, int lane,
                                                 int nthreads = 32) {
+    static_assert(M == 16 || M == 32 || M == 64, "whole halves or words per row");
     for (int r = lane; r < M; r += nthreads) {
         const unsigned long long bits = ok ? static_cast<unsigned long long>(rowbits[r]) : 0ull;
         uint32_t* row = mask + (r0 + r) * wpr;
@@ -534,12 +535,8 @@ __device__ __forceinline__ void write_mask_rows(uint32_t* mask, int64_t wpr, int
             row[c0 / 32 + 1] = static_cast<uint32_t>(bits >> 32);
         } else if constexpr (M == 32) {
             row[c0 / 32] = static_cast<uint32_t>(bits);
-        } else if constexpr (M == 16) {
-            reinterpret_cast<uint16_t*>(row)[c0 / 16] = static_cast<uint16_t>(bits);
-        } else if constexpr (M == 8) {
-            reinterpret_cast<uint8_t*>(row)[c0 / 8] = static_cast<uint8_t>(bits);
         } else {
-            if (bits) atomicOr(&row[c0 / 32], static_cast<uint32_t>(bits) << (c0 % 32));
+            reinterpret_cast<uint16_t*>(row)[c0 / 16] = static_cast<uint16_t>(bits);
         }
     }
 }
@@ -548,7 +545,7 @@ __device__ __forceinline__ void write_mask_rows(uint32_t* mask, int64_t wpr, int
 
 namespace tsenor {
 
-// Rounding of a given plan, one warp per block (M <= 32).  Entry e = r*32 + lane
+// Rounding of a given plan, one warp per block (M = 16, 32).  Entry e = r*32 + lane
 // of the block (row-major flat index) goes to this lane's register r, so the
 // loads of plan and W are coalesced along block rows.
 template <int M>

@@ -97,7 +97,7 @@ cudaError_t launch_round(const float* plan, const void* W, int64_t rows, int64_t
     const int64_t nb = (rows / M) * (cols / M);
     const int64_t wpr = (cols + 31) / 32;
     if (M == 4 || ((M == 8 || M == 16) && cols % 32)) {
-        // sub-word blocks: zero first so padding bits are 0 (and M = 4 can OR)
+        // rows narrower than a word: zero first so padding bits are 0 (and M = 4 can OR)
         cudaError_t e = cudaMemsetAsync(mask, 0, size_t(rows) * size_t(wpr) * 4, st);
         if (e != cudaSuccess) return e;
     }
