@@ -51,8 +51,12 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=15.0,
                    help="target CPU time of the bounded oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--mode", choices=["plain", "warm"], default="plain",
-                   help="warm: outer-loop re-solves with warm start and adaptive stopping (tsenor_mask_warm)")
+    p.add_argument("--mode", choices=["plain", "warm", "gap"], default="plain",
+                   help="warm: outer-loop re-solves with warm start and adaptive stopping (tsenor_mask_warm); "
+                        "gap: quality only, the GPU masks against the exact optimum on all blocks (or a "
+                        "seeded sample of --gap-blocks)")
+    p.add_argument("--gap-blocks", type=int, default=0,
+                   help="--mode gap: seeded sample size (0 = every block)")
     p.add_argument("--tol", type=float, default=1e-3, help="stop tolerance of --mode warm (nats)")
     p.add_argument("--drift", type=float, default=0.01,
                    help="--mode warm: relative change of W between consecutive outer steps")
@@ -344,6 +348,53 @@ def run_stack(args, rank, world):
         print(json.dumps(line), flush=True)
 
 
+def run_gap(args):
+    """Quality report: gap of the GPU masks to the exact (min-cost-flow) optimum, on every block of
+    the workload or on a seeded sample of whole block-rows; no timing."""
+    import torch
+    import oracle
+    import sparse_mask_search_b200 as tsl
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    if args.workload == STACK:
+        st = synth.STACK_7B_SETTINGS
+        mats = [(f"stack7b_layer0_{name}", bits, vals, st["N"], st["M"], st["tau"], st["iters"], st["sweeps"])
+                for name, bits, vals in synth.stack_7b_layer(0)]
+    else:
+        w = synth.WORKLOADS[args.workload]
+        bits, vals = synth.workload_matrix(w)
+        mats = [(w.name, bits, vals, w.N, w.M, w.tau, w.iters, w.sweeps)]
+    gaps, gaps_pruned, names = [], [], []
+    t0 = time.perf_counter()
+    for name, bits, vals, N, M, tau, iters, sweeps in mats:
+        rows, cols = vals.shape
+        Wd = to_device(bits, "bf16" if bits.dtype == np.uint16 else "f32", dev)
+        mask = tsl.tsenor_mask(Wd, N, M, tau, iters, sweeps).cpu().numpy().view(np.uint32)
+        nbr = rows // M
+        per_mat = max(1, args.gap_blocks // len(mats)) if args.gap_blocks else 0
+        if per_mat and per_mat < nbr * (cols // M):
+            k = -(-per_mat // (cols // M))                       # whole block-rows
+            sel = np.sort(synth.rng(12345).permutation(nbr)[:k])
+        else:
+            sel = np.arange(nbr)
+        rows_idx = (sel[:, None] * M + np.arange(M)[None, :]).ravel()
+        sub = np.ascontiguousarray(vals[rows_idx])
+        opt, _ = oracle.opt(sub, N, M)
+        kept = oracle.objective(sub, np.ascontiguousarray(mask[rows_idx]), N, M)
+        if np.isnan(kept).any():
+            raise RuntimeError(f"{name}: invalid GPU mask block")
+        total = oracle.blocks_view(np.abs(sub).astype(np.float64), M).sum(axis=(2, 3)).ravel()
+        gaps.append((opt - kept) / opt)
+        gaps_pruned.append((opt - kept) / np.maximum(total - opt, 1e-30))
+        names.append(f"{name}: {opt.size} blocks")
+    g, gp = np.concatenate(gaps), np.concatenate(gaps_pruned)
+    print(json.dumps({"report": "gap", "workload": args.workload, "blocks": int(g.size), "matrices": names,
+                      "mean": float(g.mean()), "max": float(g.max()), "median": float(np.median(g)),
+                      "mean_vs_pruned_mass": float(gp.mean()), "max_vs_pruned_mass": float(gp.max()),
+                      "definition": "(opt - kept)/opt per block, opt = exact min-cost-flow optimum",
+                      "host_seconds": time.perf_counter() - t0, "pages_claim": "1-10% of optimal"}), flush=True)
+
+
 def blocks_identical(mask_a, mask_b, rows, cols, M):
     """Fraction of MxM blocks on which two packed masks agree bit for bit (on the device)."""
     import torch
@@ -465,6 +516,10 @@ def main(argv=None):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return 0
+    if args.mode == "gap":
+        if rank == 0:
+            run_gap(args)
         return 0
     if args.mode == "warm" and args.workload != STACK:
         if world > 1:
