@@ -437,6 +437,15 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
     int quiet = 0;                                   // anchors in a row without a swap
     for (int sw = 0; sw < sweeps && quiet < M; ++sw) {
         for (int i = 0; i < M && quiet < M; ++i) {
+            {   // skip anchors with no positive best gain (fixed between swaps)
+                const Bits P = __ballot_sync(kFullMask, lane < M && sh.bestv[lane] > 0.f);
+                const Bits ahead = P & (~Bits(0) << i);
+                if (!ahead) { quiet += M - i; break; }
+                const int nxt = lowest_bit(ahead);
+                quiet += nxt - i;
+                i = nxt;
+                if (quiet >= M) break;
+            }
             const float best = sh.bestv[i];
             const int bp = sh.bestp[i];
             if (!(best > 0.f)) { ++quiet; continue; }
@@ -715,6 +724,16 @@ __device__ void local_search_mp(const float* a, float* Bm, float* Cm, const Roun
     int quiet = 0;                                   // anchors in a row without a swap
     for (int sw = 0; sw < sweeps && quiet < M; ++sw) {
         for (int i = 0; i < M && quiet < M; ++i) {
+            {   // skip anchors with no positive best gain (fixed between swaps)
+                const Bits P = (static_cast<Bits>(__ballot_sync(kFullMask, sh.bestv[lane + 32] > 0.f)) << 32) |
+                               __ballot_sync(kFullMask, sh.bestv[lane] > 0.f);
+                const Bits ahead = P & (~Bits(0) << i);
+                if (!ahead) { quiet += M - i; break; }
+                const int nxt = lowest_bit(ahead);
+                quiet += nxt - i;
+                i = nxt;
+                if (quiet >= M) break;
+            }
             const float best = sh.bestv[i];
             const int bp = sh.bestp[i];
             if (!(best > 0.f)) { ++quiet; continue; }
