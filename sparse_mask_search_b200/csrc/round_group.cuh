@@ -169,6 +169,15 @@ __device__ void group_local_search(const float* a, const RoundView<M>& sh, int s
     int quiet = 0;
     for (int sw = 0; sw < sweeps && quiet < M; ++sw) {
         for (int i = 0; i < M && quiet < M; ++i) {
+            {   // skip anchors with no positive best gain (fixed between swaps)
+                const unsigned P = (__ballot_sync(gmask, sh.bestv[gl] > 0.f) & gmask) >> (__ffs(gmask) - 1);
+                const unsigned ahead = P & (~0u << i);
+                if (!ahead) { quiet += M - i; break; }
+                const int nxt = __ffs(ahead) - 1;
+                quiet += nxt - i;
+                i = nxt;
+                if (quiet >= M) break;
+            }
             const float best = sh.bestv[i];
             const int bp = sh.bestp[i];
             if (!(best > 0.f)) { ++quiet; continue; }
