@@ -118,3 +118,40 @@ def test_host_pipeline_matches_device_call(rows, cols, M, N, dtype):
     out2 = tsl.tsenor_mask_host(Wd.cpu(), N, M, 20.0, 120, 4, out=torch.zeros_like(ref))
     torch.cuda.current_stream().synchronize()
     assert torch.equal(out2, ref)
+
+
+@pytest.mark.parametrize("M,N", [(8, 4), (16, 8), (32, 16), (64, 32)])
+def test_offsets_beyond_int32(M, N):
+    """A matrix of more than 2^31 elements (bf16, generated on the device from a
+    seeded generator): every block valid, and blocks at the far end of the
+    matrix equal to the oracle's."""
+    rows, cols = 65536, 32832                                # 2.15e9 elements, cols a multiple of 64
+    assert rows * cols > 2 ** 31
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1234 + M)
+    Wd = (0.02 * torch.randn((rows, cols), device="cuda", generator=g)).to(torch.bfloat16)
+    tau, iters, sweeps = 20.0, 30, 2
+    tsl.tsenor_error_count()
+    mask = tsl.tsenor_mask(Wd, N, M, tau, iters, sweeps)
+    obj = tsl.tsenor_objective(Wd, mask, N, M)
+    assert tsl.tsenor_error_count() == 0
+    assert not torch.isnan(obj).any()
+    # the last block-row and a block-row across the 2^31-element mark, against the oracle
+    for r0 in (rows - M, (2 ** 31 // cols) // M * M):
+        sub = Wd[r0:r0 + M].float().cpu().numpy()
+        m_ref, keys_ref, _ = oracle.mask(sub, N, M, tau, iters, sweeps, want_keys=True)
+        m_gpu = mask[r0:r0 + M].cpu().numpy().view(np.uint32)
+        bg, br = block_bits(m_gpu, cols, M), block_bits(m_ref, cols, M)
+        assert (bg.sum(axis=3) == N).all() and (bg.sum(axis=2) == N).all()
+        same = (bg == br).all(axis=(2, 3)).ravel()
+        if not same.all():
+            # a differing block must come from a near-tie of the oracle's keys (blocks are
+            # independent, so the plan of this block-row alone is the plan of the full solve)
+            plan = tsl.tsenor_plan(Wd[r0:r0 + M].contiguous(), N, M, tau, iters).cpu().numpy()
+            Pg, Pr = oracle.blocks_view(plan, M), oracle.blocks_view(keys_ref, M)
+            A = oracle.blocks_view(np.abs(sub), M)
+            for c in np.nonzero(~same)[0]:
+                assert max_inverted_gap(Pr[0, c], Pg[0, c], A[0, c]) <= NEAR_TIE, (r0, c)
+        assert same.mean() >= 0.99
+    del Wd, mask, obj
+    torch.cuda.empty_cache()
