@@ -58,6 +58,8 @@ def parse_args(argv=None):
     p.add_argument("--gap-blocks", type=int, default=0,
                    help="--mode gap: seeded sample size (0 = every block)")
     p.add_argument("--tol", type=float, default=1e-3, help="stop tolerance of --mode warm (nats)")
+    p.add_argument("--shape", default=None,
+                   help="ROWSxCOLS: the workload's values and settings at another shape (small profiling cases)")
     p.add_argument("--drift", type=float, default=0.01,
                    help="--mode warm: relative change of W between consecutive outer steps")
     return p.parse_args(argv)
@@ -154,6 +156,18 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(use), "samples_in_timed_region": len(inside),
                 "power_w_max": max((float(p[3]) for p in use if p[3].replace(".", "").isdigit()), default=None)}
+
+
+def workload_of(args):
+    """The named workload, at --shape ROWSxCOLS when given."""
+    w = synth.WORKLOADS[args.workload]
+    if args.shape:
+        import dataclasses
+        r, c = (int(x) for x in args.shape.lower().split("x"))
+        if r <= 0 or c <= 0 or r % w.M or c % w.M:
+            raise SystemExit(f"--shape {args.shape}: rows and cols must be positive multiples of M = {w.M}")
+        w = dataclasses.replace(w, rows=r, cols=c, name=f"{w.name}@{r}x{c}")
+    return w
 
 
 def rank_seed(w, rank: int) -> int:
@@ -339,8 +353,8 @@ def run_stack(args, rank, world):
         "roofline": {"bound": "alu", "achieved": params * iters * (1 + 2.0 / M) / (ms / 1e3) / 1e12,
                      "peak": mufu_peak_tops(SM_MAX_MHZ_FALLBACK), "unit": "TOP/s",
                      "frac": params * iters * (1 + 2.0 / M) / (ms / 1e3) / 1e12 / mufu_peak_tops(SM_MAX_MHZ_FALLBACK),
-                     "traffic": None, "kernel": "whole pass (dykstra_thread_kernel<8> + round_warp_kernel<8>)"},
-        "gpu_launches": 2 * len(mats) * args.steps,
+                     "traffic": None, "kernel": "whole pass (one fused_kernel_small<8,bf16> per matrix)"},
+        "gpu_launches": len(mats) * args.steps,
         "streams": "the 224 calls alternate between two streams (independent matrices)",
         "clocks": clocks, "cpu_baseline": None,
     }
@@ -361,7 +375,7 @@ def run_gap(args):
         mats = [(f"stack7b_layer0_{name}", bits, vals, st["N"], st["M"], st["tau"], st["iters"], st["sweeps"])
                 for name, bits, vals in synth.stack_7b_layer(0)]
     else:
-        w = synth.WORKLOADS[args.workload]
+        w = workload_of(args)
         bits, vals = synth.workload_matrix(w)
         mats = [(w.name, bits, vals, w.N, w.M, w.tau, w.iters, w.sweeps)]
     gaps, gaps_pruned, names = [], [], []
@@ -417,7 +431,7 @@ def run_warm(args, rank, world):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    w = synth.WORKLOADS[args.workload]
+    w = workload_of(args)
     storage, vals = synth.workload_matrix(w, seed=rank_seed(w, rank))
     Wa = to_device(storage, w.dtype, dev)
     g = torch.Generator(device=dev)
@@ -555,7 +569,7 @@ def main(argv=None):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    w = synth.WORKLOADS[args.workload]
+    w = workload_of(args)
     storage, vals = synth.workload_matrix(w, seed=rank_seed(w, rank))
     Wd = to_device(storage, w.dtype, dev)
     wpr = (w.cols + 31) // 32
@@ -635,16 +649,11 @@ def main(argv=None):
     value = aggregate_gparams(params, world, mean_ms_max)
     ops_per_param = w.iters * (1.0 + 2.0 / w.M)
     peak = mufu_peak_tops(SM_MAX_MHZ_FALLBACK)
-    if w.M >= 16:
-        # tsenor_mask is one fused kernel for M = 16, 32, 64: the dominant kernel
-        # is the whole step; the plan-only kernel gives the Dykstra phase alone
-        kernel_key = f"fused_kernel{w.M}<{w.dtype}>"
-        kernel_ms = mean_ms
-        launches_per_step = 1
-    else:
-        kernel_key = f"dykstra_thread_kernel<{w.M},{w.dtype}>"
-        kernel_ms = plan_ms
-        launches_per_step = 2
+    # tsenor_mask is one fused kernel per call for every M: the dominant kernel is
+    # the whole step; the plan-only kernel gives the Dykstra phase alone
+    kernel_key = f"fused_kernel{w.M}<{w.dtype}>" if w.M >= 16 else f"fused_kernel_small<{w.M},{w.dtype}>"
+    kernel_ms = mean_ms
+    launches_per_step = 1
     achieved = params * ops_per_param / (kernel_ms / 1e3) / 1e12
     traffic = profiled_traffic(kernel_key)
     line = {

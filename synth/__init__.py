@@ -62,6 +62,9 @@ WORKLOADS = {
                  16, 32, 20.0, 300, 8),
         Workload("w8192x28672_bf16_laplace_32of64", 8192, 28672, "bf16", "laplace_outliers", 0.014,
                  32, 64, 30.0, 400, 8),
+        # one matrix of the 7B-shaped stack's settings (the q projection shape, seed 0)
+        Workload("w4096x4096_bf16_normal_4of8", 4096, 4096, "bf16", "normal", 0.02,
+                 4, 8, 20.0, 200, 4),
     ]
 }
 
