@@ -104,12 +104,17 @@ struct RoundView {
 };
 
 // Per-block shared memory of the rounding steps after the sort (M <= 32).
+// The sorted order is read by the greedy only and the gain table is first
+// written by the local search, after the greedy and the repair: they share
+// their space.
 template <int M>
 struct RoundShared {
     using Bits = typename WarpRound<M>::Bits;
     static constexpr int GS = M + 1;
-    float G[M * GS];
-    uint16_t order[WarpRound<M>::EP];
+    union {
+        float G[M * GS];
+        uint16_t order[WarpRound<M>::EP];
+    };
     Bits rowbits[M];
     float bestv[M];
     int bestp[M];
