@@ -38,6 +38,17 @@ __device__ __forceinline__ float rcp_newton(float x) {
     return r;
 }
 
+// Shared-memory load of a float2 that the compiler may not move out of a
+// loop (a hoisted loop-invariant load would hold its registers for the whole
+// loop).
+__device__ __forceinline__ float2 lds_keep(const float2* p) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];"
+                 : "=f"(v.x), "=f"(v.y)
+                 : "r"(static_cast<unsigned>(__cvta_generic_to_shared(p))));
+    return v;
+}
+
 // Packed fp32 pairs (PTX f32x2, sm_100): two adds / multiplies / fmas per
 // instruction, round to nearest even per element.
 union F2U {

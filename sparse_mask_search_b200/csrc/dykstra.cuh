@@ -256,11 +256,6 @@ struct TileThread {
     __device__ __forceinline__ int col(int c) const { return C::Q * cg + lcol(c); }   // column within the block
 };
 
-// Dykstra for one block spread over its TPB threads.  On return `y` holds the
-// final state of this thread's sub-tile and `tile` the block's |W| (M x M in
-// shared memory, row stride TS).  Contains CTA-wide barriers: every thread of the CTA
-// must call it.  Returns whether the block's W is finite (false too when its
-// tile copy did not complete in time).
 // Where a block's W tile comes from.  With a tensor map (`map` non-null) the
 // tile (rows r0.., columns c0..) is copied by TMA into `raw` (M*M elements,
 // 128-byte aligned, shared memory) on the barrier `bar` and then widened to
@@ -275,38 +270,81 @@ struct TileSource {
     int64_t cols;
 };
 
+// Dykstra for one block spread over its TPB threads.  On return `out` holds the
+// plan S = 2^min(y, 0) of this thread's sub-tile.  The tile (M x M floats in
+// shared memory, row stride TS) holds the initial state y0 during the
+// iterations; with RESTORE it holds the block's |W| again on return.
+// Contains CTA-wide barriers: every thread of the CTA must call it.  Returns
+// whether the block's W is finite (false too when its tile copy did not
+// complete in time).
+//
+// The iteration is the log-space one (state y = x + log Q, base 2), kept in
+// the form y = y0 + U_i + V_j: the accumulated row and column potentials U, V
+// (fp64, in the threads that own the row or column after the reduce-scatters)
+// are the whole state.  The clipped exponentials e = 2^min(y, 0) are not
+// taken afresh every iteration: E = 2^y is carried from one iteration to the
+// next by the same update in linear form, E <- E * 2^r_i * 2^c_j (the
+// exponential of y += r_i + c_j, with r_i = log2 N - log2 R_i and
+// c_j = log2 N - log2 C_j, the very values summed into U and V), and
+// re-anchored to 2^(y0 + U + V) every kAnchorEvery iterations, so that an
+// entry that underflowed for a while recovers and the rounding of the
+// products never builds up.
+constexpr int kAnchorEvery = 64;
+
 // EXT: warm start from / export to ext.potentials of block b, stop rule
 // ext.tol2, iteration count to ext.iters_used.
-template <int M, typename T, int TS = M, bool EXT = false>
+template <int M, typename T, int TS = M, bool EXT = false, bool RESTORE = true>
 __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int64_t r0, int64_t c0, bool active,
                                                    int N, float tau, int iters, float* tile, float* colbuf,
-                                                   const TileThread<M>& th, float (&y)[4][8],
+                                                   const TileThread<M>& th, float (&out)[4][8],
                                                    const DykstraExt& ext = DykstraExt{}, int64_t b = 0) {
     using C = TileCfg<M>;
-    constexpr int P = C::P, Q = C::Q;
+    constexpr int P = C::P, Q = C::Q, Q2 = Q / 2;
+    float (&y)[P][Q] = out;                          // |W| of this thread's entries, then the plan
     const int lane = th.lane, warp = th.warp;
 
     bool loaded = true;
-    if (!src.map) {
-        // ---- 16-byte loads of the block's tile straight into |W|
-        constexpr int V = T::kVec;
-        constexpr int CPR = M / V;                 // 16-byte chunks per tile row
-        for (int q = th.t; q < M * CPR; q += C::TPB) {
-            const int i = q / CPR, v = q % CPR;
-            float tmp[V];
-            if (active) T::load16(src.W + (r0 + i) * src.cols + c0 + v * V, tmp);
-            else {
+    // |W| of the block into the tile: 16-byte loads from W, or the TMA-staged
+    // raw tile widened (zeros for an inactive block or a copy that did not land)
+    auto fill_abs = [&]() {
+        if (!src.map) {
+            constexpr int V = T::kVec;
+            constexpr int CPR = M / V;                 // 16-byte chunks per tile row
+            for (int q = th.t; q < M * CPR; q += C::TPB) {
+                const int i = q / CPR, v = q % CPR;
+                float tmp[V];
+                if (active) T::load16(src.W + (r0 + i) * src.cols + c0 + v * V, tmp);
+                else {
 #pragma unroll
-                for (int u = 0; u < V; ++u) tmp[u] = 0.f;
+                    for (int u = 0; u < V; ++u) tmp[u] = 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < V; ++u) tile[i * TS + v * V + u] = tmp[u];
             }
+        } else {
+            constexpr int V = 16 / int(sizeof(typename T::storage));   // elements per 16-byte chunk
+            constexpr int CPR = M / V;                                  // chunks per tile row
+            for (int q = th.t; q < M * CPR; q += C::TPB) {
+                const int i = q / CPR, v = q % CPR;
+                float tmp[V];
+                if (active && loaded) T::smem16(src.raw + i * M + v * V, tmp);
+                else {
 #pragma unroll
-            for (int u = 0; u < V; ++u) tile[i * TS + v * V + u] = tmp[u];
+                    for (int u = 0; u < V; ++u) tmp[u] = 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < V; ++u) tile[i * TS + v * V + u] = tmp[u];
+            }
         }
-    } else {
-        // ---- stage the block's W tile in shared memory by TMA, then |W| into the tile
+    };
+    auto block_sync = [&]() {
+        if constexpr (C::TPB <= 32) __syncwarp(); else __syncthreads();
+    };
+
+    if (src.map) {
+        // ---- stage the block's W tile in shared memory by TMA
         typename T::storage* raw = src.raw;
         uint64_t* bar = src.bar;
-        const CUtensorMap* wmap = src.map;
         // a staging address off the 128-byte grid is never handed to the copy
         // engine: the block is reported as failed instead
         const bool staged = (smem_u32(raw) & 127u) == 0 && (smem_u32(bar) & 7u) == 0;
@@ -314,30 +352,18 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
             mbar_init(bar, 1);
             mbar_init_fence();
         }
-        if constexpr (C::TPB <= 32) __syncwarp(); else __syncthreads();   // barrier initialised before any poll
+        block_sync();                                  // barrier initialised before any poll
         if (active && staged && th.t == 0) {
             mbar_arrive_expect_tx(bar, unsigned(M * M * sizeof(typename T::storage)));
-            tma_load_2d(raw, wmap, int(c0), int(r0), bar);
+            tma_load_2d(raw, src.map, int(c0), int(r0), bar);
         }
         if (active) {
             loaded = staged && mbar_wait_bounded(bar, 0);
             // a copy that did not land in time may still arrive: wait once more before the space is reused
             if (staged && !loaded) mbar_wait_bounded(bar, 0);
         }
-        constexpr int V = 16 / int(sizeof(typename T::storage));   // elements per 16-byte chunk
-        constexpr int CPR = M / V;                                  // chunks per tile row
-        for (int q = th.t; q < M * CPR; q += C::TPB) {
-            const int i = q / CPR, v = q % CPR;
-            float tmp[V];
-            if (active && loaded) T::smem16(raw + i * M + v * V, tmp);
-            else {
-#pragma unroll
-                for (int u = 0; u < V; ++u) tmp[u] = 0.f;
-            }
-#pragma unroll
-            for (int u = 0; u < V; ++u) tile[i * TS + v * V + u] = tmp[u];
-        }
     }
+    fill_abs();
     __syncthreads();
 
     float m = 0.f;
@@ -371,61 +397,88 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
         m = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
         finite = red_f[0] && red_f[1] && red_f[2] && red_f[3];
     }
+    // y0 = (x0 - tau) log2 e with x0 = tau |W| / max|W|, kept in the tile
+    // for the anchor points: column pair (k, c) of thread t at float2 slot
+    // (k * Q/2 + c) * TPB + t (consecutive threads, consecutive slots)
+    block_sync();                                    // every thread has read its |W|
     const float tau2 = tau * kLog2e;
+    float2* y0t = reinterpret_cast<float2*>(tile) + th.t;
+    static_assert(P * Q * C::TPB <= M * TS, "y0 fits the tile");
 #pragma unroll
     for (int k = 0; k < P; ++k)
 #pragma unroll
-        for (int c = 0; c < Q; ++c) {
-            const float q = m > 0.f ? __fdiv_rn(y[k][c], m) : 0.f;
-            y[k][c] = fmaf(tau2, q, -tau2);
+        for (int c = 0; c < Q2; ++c) {
+            const float q0 = m > 0.f ? __fdiv_rn(y[k][2 * c], m) : 0.f;
+            const float q1 = m > 0.f ? __fdiv_rn(y[k][2 * c + 1], m) : 0.f;
+            y0t[(k * Q2 + c) * C::TPB] = make_float2(fmaf(tau2, q0, -tau2), fmaf(tau2, q1, -tau2));
         }
-    const float fN = float(N), log2N = log2f(float(N));
+    const float log2N = log2f(float(N));
 
-    // EXT: y = y0 + U_i + V_j; this thread accumulates the potentials of the
-    // rows and columns it owns after the reduce-scatters (register k < RO
-    // holds row(k), register c < CO column col(c)).
-    // The sums are kept in fp64, so the exported state carries no
-    // accumulation error of its own.
+    // potentials of the owned rows (register k < RO holds row(k)) and columns
+    // (c < CO holds col(c)); EXT may start them from ext.potentials (nats)
     double ua[C::RO], va[C::CO];
-    if constexpr (EXT) {
-        const float* uv = (ext.warm && active) ? ext.potentials + 2 * M * b : nullptr;
-        double U[P], V[Q];
+    {
+        const float* uv = nullptr;
+        if constexpr (EXT) uv = (ext.warm && active) ? ext.potentials + 2 * M * b : nullptr;
 #pragma unroll
-        for (int k = 0; k < P; ++k) U[k] = uv ? double(uv[th.row(k)]) * kLog2eD : 0.0;
+        for (int lo = 0; lo < C::RO; ++lo) ua[lo] = uv ? double(uv[th.row(lo)]) * kLog2eD : 0.0;
 #pragma unroll
-        for (int c = 0; c < Q; ++c) V[c] = uv ? double(uv[M + th.col(c)]) * kLog2eD : 0.0;
+        for (int lo = 0; lo < C::CO; ++lo) va[lo] = uv ? double(uv[M + th.col(lo)]) * kLog2eD : 0.0;
+    }
+    // E = 2^(y0 + U_i + V_j) over this thread's entries (the potentials,
+    // rounded to fp32, all-gathered from their owners into the permuted
+    // register order)
+    float2 E2[P][Q2];                                // 2^y, column pairs packed
+    auto anchor = [&]() {
+        float U[P], V[Q];
+#pragma unroll
+        for (int lo = 0; lo < C::RO; ++lo) U[lo] = float(ua[lo]);
+#pragma unroll
+        for (int s = 1; s < C::RSR; s <<= 1)
+#pragma unroll
+            for (int hi = 0; hi < s; ++hi)
+#pragma unroll
+                for (int lo = 0; lo < C::RO; ++lo)
+                    U[(hi + s) * C::RO + lo] = __shfl_xor_sync(kFullMask, U[hi * C::RO + lo], s);
+#pragma unroll
+        for (int lo = 0; lo < C::CO; ++lo) V[lo] = float(va[lo]);
+#pragma unroll
+        for (int s = 1; s < C::RSC; s <<= 1)
+#pragma unroll
+            for (int hi = 0; hi < s; ++hi)
+#pragma unroll
+                for (int lo = 0; lo < C::CO; ++lo)
+                    V[(hi + s) * C::CO + lo] = __shfl_xor_sync(kFullMask, V[hi * C::CO + lo], s * C::CG);
 #pragma unroll
         for (int k = 0; k < P; ++k)
 #pragma unroll
-            for (int c = 0; c < Q; ++c) y[k][c] += float(U[k] + V[c]);
-#pragma unroll
-        for (int lo = 0; lo < C::RO; ++lo) ua[lo] = U[lo];
-#pragma unroll
-        for (int lo = 0; lo < C::CO; ++lo) va[lo] = V[lo];
-    }
+            for (int c = 0; c < Q2; ++c) {
+                const float2 uv2 = add2(make_float2(U[k], U[k]), make_float2(V[2 * c], V[2 * c + 1]));
+                const float2 y2 = add2(lds_keep(y0t + (k * Q2 + c) * C::TPB), uv2);
+                E2[k][c] = make_float2(ex2(y2.x), ex2(y2.y));
+            }
+    };
+    anchor();
     bool done = !finite;                             // EXT: this block has stopped
     int used = 0;
 
     // Blocks of one warp (M = 16) may differ in finiteness; all lanes run the
     // loop so that the shuffles stay converged, and a non-finite block's
     // result is discarded by the caller.
-    // Column pairs (c, c+1) of a row are handled as packed fp32x2 values.
-    constexpr int Q2 = Q / 2;
-    float2 y2[P][Q2];
-#pragma unroll
-    for (int k = 0; k < P; ++k)
-#pragma unroll
-        for (int c = 0; c < Q2; ++c) y2[k][c] = make_float2(y[k][2 * c], y[k][2 * c + 1]);
     const bool run = (C::TPB <= 32) ? (__any_sync(kFullMask, finite) != 0) : finite;
-    if (run) {
-        for (int it = 0; it < iters; ++it) {
+    bool stop = !run;
+#pragma unroll 1
+    for (int it0 = 0; it0 < iters && !stop; it0 += kAnchorEvery) {
+        if (it0 > 0) anchor();
+        const int it1 = min(iters, it0 + kAnchorEvery);
+#pragma unroll 1
+        for (int it = it0; it < it1; ++it) {
             float2 e2[P][Q2];
             float rs[P];
 #pragma unroll
             for (int k = 0; k < P; ++k) {
 #pragma unroll
-                for (int c = 0; c < Q2; ++c)
-                    e2[k][c] = make_float2(ex2(fminf(y2[k][c].x, 0.f)), ex2(fminf(y2[k][c].y, 0.f)));
+                for (int c = 0; c < Q2; ++c) e2[k][c] = make_float2(fminf(E2[k][c].x, 1.f), fminf(E2[k][c].y, 1.f));
                 const float2 acc = add2(add2(e2[k][0], e2[k][1]), add2(e2[k][2], e2[k][3]));
                 rs[k] = acc.x + acc.y;
             }
@@ -442,23 +495,21 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
 #pragma unroll
                 for (int lo = 0; lo < C::RO; ++lo)
                     rs[lo] += __shfl_xor_sync(kFullMask, rs[lo], s);
-            // owned rows: scale w = N / R and log potential r = log2 N - log2 R
-            float wv[P], rv[P];
+            // owned rows: log potential r = log2 N - log2 R and scale w = 2^r
+            float wv[P], rv[C::RO];
 #pragma unroll
             for (int lo = 0; lo < C::RO; ++lo) {
-                wv[lo] = fN * (M <= 32 ? rcp_newton(rs[lo]) : rcp(rs[lo]));   // M = 64: the MUFU form timed faster
                 rv[lo] = log2N - lg2(rs[lo]);
+                wv[lo] = ex2(rv[lo]);                // N / R_i, consistent with the potential
             }
-            // all-gather back into the permuted register order
+            // all-gather of the scales back into the permuted register order
 #pragma unroll
             for (int s = 1; s < C::RSR; s <<= 1)
 #pragma unroll
                 for (int hi = 0; hi < s; ++hi)
 #pragma unroll
-                    for (int lo = 0; lo < C::RO; ++lo) {
+                    for (int lo = 0; lo < C::RO; ++lo)
                         wv[(hi + s) * C::RO + lo] = __shfl_xor_sync(kFullMask, wv[hi * C::RO + lo], s);
-                        rv[(hi + s) * C::RO + lo] = __shfl_xor_sync(kFullMask, rv[hi * C::RO + lo], s);
-                    }
             // column partial sums of e * w
             float cs[Q];
 #pragma unroll
@@ -489,33 +540,41 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
                     cs[lo] = acc;
                 }
             }
-            float cv[Q];
+            // owned columns: log potential c = log2 N - log2 C and scale u = 2^c
+            float uv[Q], cv[C::CO];
 #pragma unroll
-            for (int lo = 0; lo < C::CO; ++lo) cv[lo] = log2N - lg2(cs[lo]);
+            for (int lo = 0; lo < C::CO; ++lo) {
+                cv[lo] = log2N - lg2(cs[lo]);
+                uv[lo] = ex2(cv[lo]);                // N / C_j
+            }
 #pragma unroll
             for (int s = 1; s < C::RSC; s <<= 1)
 #pragma unroll
                 for (int hi = 0; hi < s; ++hi)
 #pragma unroll
                     for (int lo = 0; lo < C::CO; ++lo)
-                        cv[(hi + s) * C::CO + lo] = __shfl_xor_sync(kFullMask, cv[hi * C::CO + lo], s * C::CG);
-            // y += r_i + c_j
+                        uv[(hi + s) * C::CO + lo] = __shfl_xor_sync(kFullMask, uv[hi * C::CO + lo], s * C::CG);
+            if constexpr (EXT) {
+                // a stopped block of a shared warp (M = 16) keeps its state
+                if (done) {
+#pragma unroll
+                    for (int k = 0; k < P; ++k) wv[k] = 1.f;
+#pragma unroll
+                    for (int c = 0; c < Q; ++c) uv[c] = 1.f;
+                }
+            }
+            // y += r_i + c_j, in both forms
+#pragma unroll
+            for (int k = 0; k < P; ++k)
+#pragma unroll
+                for (int c = 0; c < Q2; ++c)
+                    E2[k][c] = mul2(E2[k][c], mul2(make_float2(wv[k], wv[k]), make_float2(uv[2 * c], uv[2 * c + 1])));
             if constexpr (!EXT) {
 #pragma unroll
-                for (int k = 0; k < P; ++k)
+                for (int lo = 0; lo < C::RO; ++lo) ua[lo] += double(rv[lo]);
 #pragma unroll
-                    for (int c = 0; c < Q2; ++c)
-                        y2[k][c] = add2(y2[k][c], add2(make_float2(rv[k], rv[k]), make_float2(cv[2 * c], cv[2 * c + 1])));
+                for (int lo = 0; lo < C::CO; ++lo) va[lo] += double(cv[lo]);
             } else {
-                // a stopped block of a shared warp (M = 16) keeps its state
-                const float keep = done ? 0.f : 1.f;
-#pragma unroll
-                for (int k = 0; k < P; ++k)
-#pragma unroll
-                    for (int c = 0; c < Q2; ++c)
-                        y2[k][c] = fma2(make_float2(keep, keep),
-                                        add2(make_float2(rv[k], rv[k]), make_float2(cv[2 * c], cv[2 * c + 1])),
-                                        y2[k][c]);
                 float delta = 0.f;
 #pragma unroll
                 for (int lo = 0; lo < C::RO; ++lo) {
@@ -541,12 +600,19 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
                         all_small = __syncthreads_and(small);
                     }
                     done = done || all_small;
-                    const bool stop = (C::TPB <= 32) ? (__all_sync(kFullMask, done) != 0) : done;
+                    stop = (C::TPB <= 32) ? (__all_sync(kFullMask, done) != 0) : done;
                     if (stop) break;
                 }
             }
         }
     }
+#pragma unroll
+    for (int k = 0; k < P; ++k)
+#pragma unroll
+        for (int c = 0; c < Q2; ++c) {
+            y[k][2 * c] = fminf(E2[k][c].x, 1.f);
+            y[k][2 * c + 1] = fminf(E2[k][c].y, 1.f);
+        }
     if constexpr (EXT) {
         if (active) {
             if (ext.potentials) {
@@ -562,13 +628,11 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
             if (ext.iters_used && th.t == 0) ext.iters_used[b] = finite ? used : 0;
         }
     }
-#pragma unroll
-    for (int k = 0; k < P; ++k)
-#pragma unroll
-        for (int c = 0; c < Q2; ++c) {
-            y[k][2 * c] = y2[k][c].x;
-            y[k][2 * c + 1] = y2[k][c].y;
-        }
+    if constexpr (RESTORE) {
+        block_sync();                                // every thread has read its y0
+        fill_abs();
+        block_sync();
+    }
     return finite;
 }
 
@@ -585,7 +649,7 @@ struct PlanSmem {
 };
 
 template <int M, typename T, bool EXT = false>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 5)
 dykstra_tile_kernel(const __grid_constant__ CUtensorMap wmap, int64_t cols, int64_t n_blocks,
                     int N, float tau, int iters, float* __restrict__ plan, DykstraExt ext = {}) {
     using C = TileCfg<M>;
@@ -601,9 +665,9 @@ dykstra_tile_kernel(const __grid_constant__ CUtensorMap wmap, int64_t cols, int6
     const int64_t nbc = cols / M;
     const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
 
-    float y[C::P][C::Q];
+    float S[C::P][C::Q];                      // plan of this thread's entries
     const TileSource<T> src{&wmap, raw, bar, nullptr, 0};
-    const bool finite = dykstra_tile_solve<M, T, M, EXT>(src, r0, c0, active, N, tau, iters, tile, colbuf, th, y, ext,
+    const bool finite = dykstra_tile_solve<M, T, M, EXT, false>(src, r0, c0, active, N, tau, iters, tile, colbuf, th, S, ext,
                                                          b);
 
     // ---- plan via the smem tile, then 16-byte coalesced stores
@@ -612,7 +676,7 @@ dykstra_tile_kernel(const __grid_constant__ CUtensorMap wmap, int64_t cols, int6
     for (int k = 0; k < C::P; ++k)
 #pragma unroll
         for (int c = 0; c < C::Q; ++c)
-            tile[th.row(k) * M + th.col(c)] = finite ? plan_value(y[k][c]) : __int_as_float(0x7fc00000);
+            tile[th.row(k) * M + th.col(c)] = finite ? S[k][c] : __int_as_float(0x7fc00000);
     __syncthreads();
     if (active) {
         constexpr int CPR = M / 4;

@@ -19,16 +19,15 @@
 
 namespace tsenor {
 
-// bf16: registers capped at 80 (the bound for 6 CTAs per SM; shared memory
-// still admits 5, so only the generated code changes): 4.98 ms against 5.01 ms
-// with the 96-register cap of 5 CTAs and 5.03 ms uncapped on the 4096x11008
-// 16:32 workload, in two runs each.  The fp32 key needs more registers; the
-// EXT instance keeps the 96-register cap.
+// bf16: registers capped at 96, five CTAs per SM (shared memory would admit
+// six): 4.01 ms against 4.06 ms with the 80-register cap of six CTAs on the
+// 4096x11008 16:32 workload.  The fp32 key needs more registers.
 // The tile is read with 16-byte loads here, not staged by TMA: on the same
 // workload the TMA-staged variant of this kernel timed 5.16 ms against
-// 5.01 ms (the plan kernel of the same M gained 0.7% from TMA staging).
+// 5.01 ms with the earlier exponential-per-iteration solver (the plan kernel
+// of the same M gained 0.7% from TMA staging).
 template <typename T, bool EXT = false>
-__global__ void __launch_bounds__(128, std::is_same<T, BF16>::value ? (EXT ? 5 : 6) : 4)
+__global__ void __launch_bounds__(128, std::is_same<T, BF16>::value ? 5 : 4)
 fused_kernel32(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
                int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr, DykstraExt ext = {}) {
     constexpr int M = 32;
@@ -45,9 +44,9 @@ fused_kernel32(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
     const int64_t nbc = cols / M;
     const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
 
-    float y[C::P][C::Q];
+    float S[C::P][C::Q];                      // plan of this thread's entries
     const TileSource<T> src{nullptr, nullptr, nullptr, W, cols};
-    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(src, r0, c0, active, N, tau, iters, tile, nullptr, th, y,
+    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(src, r0, c0, active, N, tau, iters, tile, nullptr, th, S,
                                                           ext, b);
     if (!active) return;                              // no CTA-wide barrier follows
 
@@ -57,7 +56,7 @@ fused_kernel32(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
 #pragma unroll
         for (int c = 0; c < C::Q; ++c) {
             const int e = th.row(k) * M + th.col(c);
-            key[k * C::Q + c] = Key::make(plan_value(y[k][c]), tile[th.row(k) * TS + th.col(c)], e);
+            key[k * C::Q + c] = Key::make(S[k][c], tile[th.row(k) * TS + th.col(c)], e);
         }
     bool ok = finite;                                 // one block per warp: uniform
     if (ok) ok = round_block_warp<M, Key>(key, tile, shs[th.blk].view(), N, sweeps, th.lane);
@@ -72,7 +71,7 @@ constexpr size_t fused32_smem() {
 
 // M = 16: a warp holds 4 blocks of 8 threads each.
 template <typename T, bool EXT = false>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 5)
 fused_kernel16(const __grid_constant__ CUtensorMap wmap, int64_t cols, int64_t n_blocks, int N, float tau,
                int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr, DykstraExt ext = {}) {
     constexpr int M = 16, TS = M + 1, E = M * M;
@@ -94,16 +93,16 @@ fused_kernel16(const __grid_constant__ CUtensorMap wmap, int64_t cols, int64_t n
     const int64_t nbc = cols / M;
     const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
 
-    float y[C::P][C::Q];
+    float S[C::P][C::Q];                      // plan of this thread's entries
     const TileSource<T> src{&wmap, reinterpret_cast<typename T::storage*>(ptiles + th.blk * E), bars + th.blk,
                             nullptr, 0};
-    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(src, r0, c0, active, N, tau, iters, tile, nullptr, th, y,
+    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(src, r0, c0, active, N, tau, iters, tile, nullptr, th, S,
                                                           ext, b);
     float* ptile = ptiles + th.blk * E;
 #pragma unroll
     for (int k = 0; k < C::P; ++k)
 #pragma unroll
-        for (int c = 0; c < C::Q; ++c) ptile[th.row(k) * M + th.col(c)] = plan_value(y[k][c]);
+        for (int c = 0; c < C::Q; ++c) ptile[th.row(k) * M + th.col(c)] = S[k][c];
     if (th.t == 0) flags[th.blk] = finite;
     __syncwarp();
 
@@ -220,7 +219,7 @@ fused_kernel_small(const typename T::storage* __restrict__ W, int64_t cols, int6
 static_assert(Round64Smem<KeyB>::kColbufFloats >= 2 * 4 * 32 * TileCfg<64>::CO, "column-sum buffer");
 
 template <typename T, bool EXT = false>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, std::is_same<T, BF16>::value ? 4 : 1)
 fused_kernel64(const __grid_constant__ CUtensorMap wmap, int64_t cols, int64_t n_blocks, int N, float tau,
                int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr, DykstraExt ext = {}) {
     constexpr int M = 64, TS = M + 1;
@@ -236,10 +235,10 @@ fused_kernel64(const __grid_constant__ CUtensorMap wmap, int64_t cols, int64_t n
     const int64_t nbc = cols / M;
     const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
 
-    float y[C::P][C::Q];
+    float S[C::P][C::Q];                      // plan of this thread's entries
     // the raw W tile is staged in the sort exchange space
     const TileSource<T> src{&wmap, reinterpret_cast<typename T::storage*>(&sm.u), &sm.tma_bar, nullptr, 0};
-    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(src, r0, c0, true, N, tau, iters, sm.a, sm.v.colbuf, th, y,
+    const bool finite = dykstra_tile_solve<M, T, TS, EXT>(src, r0, c0, true, N, tau, iters, sm.a, sm.v.colbuf, th, S,
                                                           ext, b);
     Key key[C::P * C::Q];
 #pragma unroll
@@ -247,7 +246,7 @@ fused_kernel64(const __grid_constant__ CUtensorMap wmap, int64_t cols, int64_t n
 #pragma unroll
         for (int c = 0; c < C::Q; ++c) {
             const int row = th.row(k), col = th.col(c);
-            key[k * C::Q + c] = Key::make(plan_value(y[k][c]), sm.a[row * TS + col], row * M + col);
+            key[k * C::Q + c] = Key::make(S[k][c], sm.a[row * TS + col], row * M + col);
         }
     bool ok = finite;                                   // uniform over the CTA
     if (ok) ok = round_block_cta64(key, sm, N, sweeps, th.tid);
