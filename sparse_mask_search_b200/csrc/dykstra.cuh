@@ -27,6 +27,8 @@
 //    plain solve.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "tma.cuh"
 
@@ -44,20 +46,40 @@ struct DykstraExt {
     int warm;               // nonzero: start from `potentials`
 };
 
-// Plan entry of one state value: S = 2^min(y, 0), exactly 1 when clipped.
-__device__ __forceinline__ float plan_value(float y) { return y >= 0.f ? 1.f : ex2(y); }
+// Iterations between two anchor points of the linear-form exponentials
+// (see dykstra_tile_solve).
+constexpr int kAnchorEvery = 64;
+
 
 // ---------------------------------------------------------------------------
 // M = 4, 8: one thread holds a whole block in registers.  Rows are streamed:
 // the exponentials of one row live only until its column contributions are
 // added, so no cross-thread traffic is needed at all.
 // ---------------------------------------------------------------------------
-// Dykstra for block b (rows r0.., columns c0..) by one thread.  On return y
-// holds the final state; returns whether the block's W is finite.
+// Shared-memory load of a float4 that the compiler may not move out of a loop.
+__device__ __forceinline__ float4 lds4_keep(const float* p) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(static_cast<unsigned>(__cvta_generic_to_shared(p))));
+    return v;
+}
+
+// Dykstra for block b (rows r0.., columns c0..) by one thread, in the form of
+// dykstra_tile_solve: the state is y = y0 + U_i + V_j, E = 2^y is carried in
+// linear form between anchor points (E *= 2^r_i after row i's step,
+// E *= 2^c_j after the column step) and recomputed from y0 + U + V every
+// kAnchorEvery iterations.  y0s: this thread's M*M floats of shared memory
+// (16-byte aligned), which hold y0 during the iterations.  On return `s`
+// holds the plan 2^min(y, 0); returns whether the block's W is finite.
+// The potentials are summed in fp32 (fp64 for EXT, whose exported state
+// must carry no accumulation error of its own).
 template <int M, typename T, bool EXT = false>
 __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* __restrict__ W, int64_t cols,
                                                      int64_t b, int64_t r0, int64_t c0, int N, float tau,
-                                                     int iters, const DykstraExt& ext, float (&y)[M][M]) {
+                                                     int iters, const DykstraExt& ext, float (&s)[M][M],
+                                                     float* y0s) {
+    float (&y)[M][M] = s;                            // |W|, then y0, then the plan
 #pragma unroll
     for (int i = 0; i < M; ++i) {
         const typename T::storage* src = W + (r0 + i) * cols + c0;
@@ -80,40 +102,55 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
         }
     const float tau2 = tau * kLog2e;
 #pragma unroll
-    for (int i = 0; i < M; ++i)
+    for (int i = 0; i < M; ++i) {
 #pragma unroll
         for (int j = 0; j < M; ++j) {
             const float q = m > 0.f ? __fdiv_rn(y[i][j], m) : 0.f;
             y[i][j] = fmaf(tau2, q, -tau2);
         }
-    const float fN = float(N), log2N = log2f(float(N));
+#pragma unroll
+        for (int v = 0; v < M / 4; ++v)
+            reinterpret_cast<float4*>(y0s + i * M)[v] = make_float4(y[i][4 * v], y[i][4 * v + 1], y[i][4 * v + 2],
+                                                                    y[i][4 * v + 3]);
+    }
+    const float log2N = log2f(float(N));
 
-    // EXT: accumulated potentials in log2 units, summed in fp64 so that the
-    // exported state carries no accumulation error of its own
-    double U[M], V[M];
+    using Acc = double;
+    Acc U[M], V[M];                                  // accumulated potentials, log2 units
     int used = 0;
-    if constexpr (EXT) {
-        const float* uv = ext.warm ? ext.potentials + 2 * M * b : nullptr;
+    {
+        const float* uv = nullptr;
+        if constexpr (EXT) uv = ext.warm ? ext.potentials + 2 * M * b : nullptr;
 #pragma unroll
         for (int k = 0; k < M; ++k) {
-            U[k] = uv ? double(uv[k]) * kLog2eD : 0.0;
-            V[k] = uv ? double(uv[M + k]) * kLog2eD : 0.0;
+            U[k] = uv ? Acc(double(uv[k]) * kLog2eD) : Acc(0);
+            V[k] = uv ? Acc(double(uv[M + k]) * kLog2eD) : Acc(0);
         }
+    }
+    // column pairs (j, j+1) as packed fp32x2 values
+    constexpr int M2 = M / 2;
+    float2 E2[M][M2];
+    auto anchor = [&]() {
 #pragma unroll
         for (int i = 0; i < M; ++i)
 #pragma unroll
-            for (int j = 0; j < M; ++j) y[i][j] += float(U[i] + V[j]);
-    }
-
-    // column pairs (j, j+1) as packed fp32x2 values
-    constexpr int M2 = M / 2;
-    float2 y2[M][M2];
-#pragma unroll
-    for (int i = 0; i < M; ++i)
-#pragma unroll
-        for (int c = 0; c < M2; ++c) y2[i][c] = make_float2(y[i][2 * c], y[i][2 * c + 1]);
-    if (finite) {
-        for (int t = 0; t < iters; ++t) {
+            for (int v = 0; v < M / 4; ++v) {
+                const float4 q = lds4_keep(y0s + i * M + 4 * v);
+                const float u = float(U[i]);
+                const float2 a = add2(make_float2(q.x, q.y), add2(make_float2(u, u), make_float2(float(V[4 * v]), float(V[4 * v + 1]))));
+                const float2 c = add2(make_float2(q.z, q.w), add2(make_float2(u, u), make_float2(float(V[4 * v + 2]), float(V[4 * v + 3]))));
+                E2[i][2 * v] = make_float2(ex2(a.x), ex2(a.y));
+                E2[i][2 * v + 1] = make_float2(ex2(c.x), ex2(c.y));
+            }
+    };
+    anchor();
+    bool stop = !finite;
+#pragma unroll 1
+    for (int t0 = 0; t0 < iters && !stop; t0 += kAnchorEvery) {
+        if (t0 > 0) anchor();
+        const int t1 = min(iters, t0 + kAnchorEvery);
+#pragma unroll 1
+        for (int t = t0; t < t1; ++t) {
             float delta = 0.f;                         // largest |r_i|, |c_j| of this iteration (EXT)
             float2 C2[M2];
 #pragma unroll
@@ -122,36 +159,34 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
             for (int i = 0; i < M; ++i) {
                 float2 e2[M2];
 #pragma unroll
-                for (int c = 0; c < M2; ++c)
-                    e2[c] = make_float2(ex2(fminf(y2[i][c].x, 0.f)), ex2(fminf(y2[i][c].y, 0.f)));
+                for (int c = 0; c < M2; ++c) e2[c] = make_float2(fminf(E2[i][c].x, 1.f), fminf(E2[i][c].y, 1.f));
                 float2 acc = e2[0];
 #pragma unroll
                 for (int c = 1; c < M2; ++c) acc = add2(acc, e2[c]);
-                const float R = acc.x + acc.y;
-                const float w = fN * rcp_newton(R);
-                const float r = log2N - lg2(R);
-                const float2 w2 = make_float2(w, w), r2 = make_float2(r, r);
+                const float r = log2N - lg2(acc.x + acc.y);
+                const float w = ex2(r);                  // N / R_i
+                const float2 w2 = make_float2(w, w);
 #pragma unroll
                 for (int c = 0; c < M2; ++c) {
                     C2[c] = fma2(e2[c], w2, C2[c]);
-                    y2[i][c] = add2(y2[i][c], r2);
+                    E2[i][c] = mul2(E2[i][c], w2);
                 }
-                if constexpr (EXT) { U[i] += double(r); delta = fmaxf(delta, fabsf(r)); }
+                U[i] += Acc(r);
+                if constexpr (EXT) delta = fmaxf(delta, fabsf(r));
             }
 #pragma unroll
             for (int c = 0; c < M2; ++c) {
                 const float2 cv = make_float2(log2N - lg2(C2[c].x), log2N - lg2(C2[c].y));
+                const float2 u2 = make_float2(ex2(cv.x), ex2(cv.y));   // N / C_j
 #pragma unroll
-                for (int i = 0; i < M; ++i) y2[i][c] = add2(y2[i][c], cv);
-                if constexpr (EXT) {
-                    V[2 * c] += double(cv.x);
-                    V[2 * c + 1] += double(cv.y);
-                    delta = fmaxf(delta, fmaxf(fabsf(cv.x), fabsf(cv.y)));
-                }
+                for (int i = 0; i < M; ++i) E2[i][c] = mul2(E2[i][c], u2);
+                V[2 * c] += Acc(cv.x);
+                V[2 * c + 1] += Acc(cv.y);
+                if constexpr (EXT) delta = fmaxf(delta, fmaxf(fabsf(cv.x), fabsf(cv.y)));
             }
             used = t + 1;
             if constexpr (EXT) {
-                if (ext.tol2 > 0.f && delta <= ext.tol2) break;
+                if (ext.tol2 > 0.f && delta <= ext.tol2) { stop = true; break; }
             }
         }
     }
@@ -159,8 +194,8 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
     for (int i = 0; i < M; ++i)
 #pragma unroll
         for (int c = 0; c < M2; ++c) {
-            y[i][2 * c] = y2[i][c].x;
-            y[i][2 * c + 1] = y2[i][c].y;
+            y[i][2 * c] = fminf(E2[i][c].x, 1.f);
+            y[i][2 * c + 1] = fminf(E2[i][c].y, 1.f);
         }
     if constexpr (EXT) {
         if (ext.potentials) {
@@ -176,26 +211,32 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
     return finite;
 }
 
+// Per-thread y0 space of dykstra_thread_kernel (floats; padded so that the
+// threads' 16-byte accesses do not share banks).
+template <int M>
+__host__ __device__ constexpr int thread_y0_stride() { return M * M + 4; }
+
 template <int M, typename T, bool EXT = false>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 4)
 dykstra_thread_kernel(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks,
                       int N, float tau, int iters, float* __restrict__ plan, DykstraExt ext = {}) {
+    extern __shared__ __align__(16) float thread_y0[];
     const int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
     if (b >= n_blocks) return;
     const int64_t nbc = cols / M;
     const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
-    float y[M][M];
-    const bool finite = dykstra_thread_solve<M, T, EXT>(W, cols, b, r0, c0, N, tau, iters, ext, y);
+    float S[M][M];
+    const bool finite = dykstra_thread_solve<M, T, EXT>(W, cols, b, r0, c0, N, tau, iters, ext, S,
+                                                        thread_y0 + threadIdx.x * thread_y0_stride<M>());
 #pragma unroll
     for (int i = 0; i < M; ++i) {
-        float s[M];
-#pragma unroll
-        for (int j = 0; j < M; ++j)
-            s[j] = !finite ? __int_as_float(0x7fc00000) : plan_value(y[i][j]);
         float* dst = plan + (r0 + i) * cols + c0;
 #pragma unroll
         for (int v = 0; v < M / 4; ++v)
-            reinterpret_cast<float4*>(dst)[v] = make_float4(s[4 * v], s[4 * v + 1], s[4 * v + 2], s[4 * v + 3]);
+            reinterpret_cast<float4*>(dst)[v] =
+                finite ? make_float4(S[i][4 * v], S[i][4 * v + 1], S[i][4 * v + 2], S[i][4 * v + 3])
+                       : make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
+                                     __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
     }
 }
 
@@ -289,7 +330,6 @@ struct TileSource {
 // re-anchored to 2^(y0 + U + V) every kAnchorEvery iterations, so that an
 // entry that underflowed for a while recovers and the rounding of the
 // products never builds up.
-constexpr int kAnchorEvery = 64;
 
 // EXT: warm start from / export to ext.potentials of block b, stop rule
 // ext.tol2, iteration count to ext.iters_used.

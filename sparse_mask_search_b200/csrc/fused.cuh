@@ -153,7 +153,7 @@ struct FusedSmallCfg {
 };
 
 template <int M, typename T, bool EXT = false>
-__global__ void __launch_bounds__(64)
+__global__ void __maxnreg__(128)
 fused_kernel_small(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
                    int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr, DykstraExt ext = {}) {
     using Cfg = FusedSmallCfg<M>;
@@ -169,16 +169,15 @@ fused_kernel_small(const typename T::storage* __restrict__ W, int64_t cols, int6
         const int64_t b = int64_t(blockIdx.x) * Cfg::THREADS + t;
         if (b < n_blocks) {
             const int64_t r0 = (b / nbc) * M, c0 = (b % nbc) * M;
-            float y[M][M];
-            const bool finite = dykstra_thread_solve<M, T, EXT>(W, cols, b, r0, c0, N, tau, iters, ext, y);
-            float* dst = plans + t * Cfg::SS;
+            float S[M][M];                                    // plan of the block
+            float* dst = plans + t * Cfg::SS;                 // y0 during the solve, then the plan
+            const bool finite = dykstra_thread_solve<M, T, EXT>(W, cols, b, r0, c0, N, tau, iters, ext, S, dst);
 #pragma unroll
             for (int i = 0; i < M; ++i)
 #pragma unroll
                 for (int v = 0; v < M / 4; ++v)
                     reinterpret_cast<float4*>(dst + i * M)[v] =
-                        make_float4(plan_value(y[i][4 * v]), plan_value(y[i][4 * v + 1]),
-                                    plan_value(y[i][4 * v + 2]), plan_value(y[i][4 * v + 3]));
+                        make_float4(S[i][4 * v], S[i][4 * v + 1], S[i][4 * v + 2], S[i][4 * v + 3]);
             flags[t] = finite;
         }
     }

@@ -75,7 +75,10 @@ cudaError_t launch_plan(const void* W, int64_t rows, int64_t cols, int N, float 
     const auto* w = static_cast<const typename T::storage*>(W);
     if constexpr (M <= 8) {
         const int64_t grid = (nb + 127) / 128;
-        dykstra_thread_kernel<M, T, EXT><<<dim3(unsigned(grid)), 128, 0, st>>>(w, cols, nb, N, tau, iters, plan, ext);
+        constexpr size_t smem = sizeof(float) * 128 * thread_y0_stride<M>();
+        static_assert(smem <= 48 * 1024, "default dynamic shared memory limit");
+        dykstra_thread_kernel<M, T, EXT><<<dim3(unsigned(grid)), 128, smem, st>>>(w, cols, nb, N, tau, iters, plan,
+                                                                                   ext);
     } else {
         CUtensorMap map;
         cudaError_t e = encode_w_map<T>(&map, W, rows, cols, M);
