@@ -35,7 +35,11 @@ DEFAULT_WORKLOAD = "w4096x11008_bf16_t3_16of32"
 METRIC = "transposable N:M mask Gparams/s at 1 B200 (% of roofline); mean gap to exact opt"
 STACK = "stack7b"                  # 32 layers x 7 matrices, 4:8, one pass = one step
 SM_COUNT = 148
-MUFU_PER_CLK_PER_SM = 16          # ex2 / lg2 / rcp results per clock per SM
+FP32_LANES_PER_CLK_PER_SM = 128   # fp32 add / mul / fma results per clock per SM (FMA pipe)
+# Algorithmic FMA-pipe work of one Dykstra iteration per entry: the row-sum
+# add, the column-sum fma and the row and column scalings of E (the clip
+# min(E, 1) runs on the ALU pipe and is not counted).
+FP32_OPS_PER_ENTRY_ITER = 4
 SM_MAX_MHZ_FALLBACK = 1965.0
 L2_FLUSH_BYTES = 256 << 20
 
@@ -75,8 +79,11 @@ def measured_peaks():
         return {}
 
 
-def mufu_peak_tops(sm_mhz):
-    return SM_COUNT * MUFU_PER_CLK_PER_SM * sm_mhz * 1e6 / 1e12
+def fp32_peak_tops(sm_mhz):
+    return SM_COUNT * FP32_LANES_PER_CLK_PER_SM * sm_mhz * 1e6 / 1e12
+
+
+PEAK_BASIS = f"{SM_COUNT} SMs x {FP32_LANES_PER_CLK_PER_SM} FP32 lanes/clk x {SM_MAX_MHZ_FALLBACK:.0f} MHz"
 
 
 def source_digest():
@@ -350,10 +357,12 @@ def run_stack(args, rank, world):
                    "iters": iters, "sweeps": sweeps,
                    "l2": "inputs larger than L2 (13 GB per pass, each matrix read once per pass)",
                    "total_wall_s_per_pass": ms_max / 1e3, "host_generation_s": t_gen},
-        "roofline": {"bound": "alu", "achieved": params * iters * (1 + 2.0 / M) / (ms / 1e3) / 1e12,
-                     "peak": mufu_peak_tops(SM_MAX_MHZ_FALLBACK), "unit": "TOP/s",
-                     "frac": params * iters * (1 + 2.0 / M) / (ms / 1e3) / 1e12 / mufu_peak_tops(SM_MAX_MHZ_FALLBACK),
-                     "traffic": None, "kernel": "whole pass (one fused_kernel_small<8,bf16> per matrix)"},
+        "roofline": {"bound": "alu", "achieved": params * iters * FP32_OPS_PER_ENTRY_ITER / (ms / 1e3) / 1e12,
+                     "peak": fp32_peak_tops(SM_MAX_MHZ_FALLBACK), "unit": "TOP/s",
+                     "frac": params * iters * FP32_OPS_PER_ENTRY_ITER / (ms / 1e3) / 1e12
+                     / fp32_peak_tops(SM_MAX_MHZ_FALLBACK),
+                     "traffic": None, "kernel": "whole pass (one fused_kernel_small<8,bf16> per matrix)",
+                     "ops": f"{FP32_OPS_PER_ENTRY_ITER} FP32 ops per entry and iteration x T", "peak_basis": PEAK_BASIS},
         "gpu_launches": len(mats) * args.steps,
         "streams": "the 224 calls alternate between two streams (independent matrices)",
         "clocks": clocks, "cpu_baseline": None,
@@ -496,8 +505,8 @@ def run_warm(args, rank, world):
     plain_ms = statistics.mean(a.elapsed_time(b) for a, b in pev)
     tsl.tsenor_error_count()
     params = w.rows * w.cols
-    ops = params * mean_iters * (1.0 + 2.0 / w.M)
-    peak = mufu_peak_tops(SM_MAX_MHZ_FALLBACK)
+    ops = params * mean_iters * FP32_OPS_PER_ENTRY_ITER
+    peak = fp32_peak_tops(SM_MAX_MHZ_FALLBACK)
     line = {
         "metric": METRIC,
         "value": aggregate_gparams(params, world, ms_max), "unit": "Gparams/s", "n_gpus": world,
@@ -513,7 +522,8 @@ def run_warm(args, rank, world):
         "roofline": {"bound": "alu", "achieved": ops / (ms / 1e3) / 1e12, "peak": peak, "unit": "TOP/s",
                      "frac": ops / (ms / 1e3) / 1e12 / peak, "traffic": None,
                      "kernel": f"fused_kernel{w.M}<{w.dtype},EXT>" if w.M >= 16 else "plan + round",
-                     "ops": "mean iterations run x (1+2/M) MUFU ops per param"},
+                     "ops": f"mean iterations run x {FP32_OPS_PER_ENTRY_ITER} FP32 ops per param",
+                     "peak_basis": PEAK_BASIS},
         "gpu_launches": (1 if w.M >= 16 else 2) * args.steps,
         "clocks": clocks, "cpu_baseline": None, "e2e": None,
     }
@@ -647,8 +657,8 @@ def main(argv=None):
 
     params = w.rows * w.cols
     value = aggregate_gparams(params, world, mean_ms_max)
-    ops_per_param = w.iters * (1.0 + 2.0 / w.M)
-    peak = mufu_peak_tops(SM_MAX_MHZ_FALLBACK)
+    ops_per_param = w.iters * FP32_OPS_PER_ENTRY_ITER
+    peak = fp32_peak_tops(SM_MAX_MHZ_FALLBACK)
     # tsenor_mask is one fused kernel per call for every M: the dominant kernel is
     # the whole step; the plan-only kernel gives the Dykstra phase alone
     kernel_key = f"fused_kernel{w.M}<{w.dtype}>" if w.M >= 16 else f"fused_kernel_small<{w.M},{w.dtype}>"
@@ -667,8 +677,9 @@ def main(argv=None):
                    "parallelism": f"replicas x{world}: each rank solves its own matrix, no collective"},
         "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TOP/s",
                      "frac": achieved / peak, "traffic": traffic, "kernel": kernel_key,
-                     "ops": f"{ops_per_param:.2f} MUFU ops (ex2/lg2) per param = T*(1+2/M)",
-                     "peak_basis": f"{SM_COUNT} SMs x {MUFU_PER_CLK_PER_SM} MUFU/clk x {SM_MAX_MHZ_FALLBACK:.0f} MHz",
+                     "ops": f"{ops_per_param:.0f} FP32 ops per param = T x {FP32_OPS_PER_ENTRY_ITER} (row-sum add, "
+                            "column-sum fma, row and column scaling of E per entry and iteration)",
+                     "peak_basis": PEAK_BASIS,
                      "kernel_ms": kernel_ms},
         "breakdown_ms": {"dykstra_plan_kernel_alone": plan_ms, "rest_of_step": round_ms,
                          "dykstra_frac_of_peak": params * ops_per_param / (plan_ms / 1e3) / 1e12 / peak},

@@ -8,7 +8,7 @@ namespace tsenor {
 
 constexpr unsigned kFullMask = 0xffffffffu;
 
-// Hardware base-2 exponential / logarithm / reciprocal (PTX approx forms, MUFU).
+// Hardware base-2 exponential / logarithm (PTX approx forms, MUFU).
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -19,25 +19,6 @@ __device__ __forceinline__ float lg2(float x) {
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-__device__ __forceinline__ float rcp(float x) {
-    float y;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// 1/x on the FMA pipe: a bit-pattern first guess (x0 = bits^-1(K - bits(x)),
-// K chosen here to minimise the worst relative error of x0 over [1, 2): 5.1%)
-// refined by three Newton steps x <- x + x (1 - x*a); worst relative error
-// 6e-8 for normal positive x.  Used where a reciprocal would otherwise take a
-// MUFU slot that the exponentials need.
-__device__ __forceinline__ float rcp_newton(float x) {
-    float r = __int_as_float(0x7EF311C0 - __float_as_int(x));
-    r = fmaf(r, fmaf(-x, r, 1.f), r);
-    r = fmaf(r, fmaf(-x, r, 1.f), r);
-    r = fmaf(r, fmaf(-x, r, 1.f), r);
-    return r;
-}
-
 // Shared-memory load of a float2 that the compiler may not move out of a
 // loop (a hoisted loop-invariant load would hold its registers for the whole
 // loop).
