@@ -8,7 +8,7 @@ namespace tsenor {
 
 constexpr unsigned kFullMask = 0xffffffffu;
 
-// Hardware base-2 exponential / logarithm (PTX approx forms, MUFU).
+// Hardware base-2 exponential / logarithm / reciprocal (PTX approx forms, MUFU).
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -17,6 +17,11 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ float lg2(float x) {
     float y;
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 // Shared-memory load of a float2 that the compiler may not move out of a

@@ -69,11 +69,13 @@ __device__ __forceinline__ float4 lds4_keep(const float* p) {
 // dykstra_tile_solve: the state is y = y0 + U_i + V_j, E = 2^y is carried in
 // linear form between anchor points (E *= 2^r_i after row i's step,
 // E *= 2^c_j after the column step) and recomputed from y0 + U + V every
-// kAnchorEvery iterations.  y0s: this thread's M*M floats of shared memory
-// (16-byte aligned), which hold y0 during the iterations.  On return `s`
-// holds the plan 2^min(y, 0); returns whether the block's W is finite.
-// The potentials are summed in fp32 (fp64 for EXT, whose exported state
-// must carry no accumulation error of its own).
+// kAnchorEvery iterations.  The scalings are N / R_i and N / C_j by the
+// hardware reciprocal; their products since the last anchor point are kept
+// per row and column and their base-2 logarithms added to U and V (fp32) at
+// the next one, so the potentials follow the very factors applied to E.
+// y0s: this thread's M*M floats of shared memory (16-byte aligned), which
+// hold y0 during the iterations.  On return `s` holds the plan
+// 2^min(y, 0); returns whether the block's W is finite.
 template <int M, typename T, bool EXT = false>
 __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* __restrict__ W, int64_t cols,
                                                      int64_t b, int64_t r0, int64_t c0, int N, float tau,
@@ -113,32 +115,46 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
             reinterpret_cast<float4*>(y0s + i * M)[v] = make_float4(y[i][4 * v], y[i][4 * v + 1], y[i][4 * v + 2],
                                                                     y[i][4 * v + 3]);
     }
-    const float log2N = log2f(float(N));
+    const float fN = float(N);
 
-    using Acc = double;
-    Acc U[M], V[M];                                  // accumulated potentials, log2 units
+    // potentials (log2 units) as of the last anchor point, and the products of
+    // the row and column scalings applied since then (their logarithms are
+    // added at the next anchor point)
+    float U[M], V[M], PU[M], PV[M];
     int used = 0;
     {
         const float* uv = nullptr;
         if constexpr (EXT) uv = ext.warm ? ext.potentials + 2 * M * b : nullptr;
 #pragma unroll
         for (int k = 0; k < M; ++k) {
-            U[k] = uv ? Acc(double(uv[k]) * kLog2eD) : Acc(0);
-            V[k] = uv ? Acc(double(uv[M + k]) * kLog2eD) : Acc(0);
+            U[k] = uv ? float(double(uv[k]) * kLog2eD) : 0.f;
+            V[k] = uv ? float(double(uv[M + k]) * kLog2eD) : 0.f;
+            PU[k] = 1.f;
+            PV[k] = 1.f;
         }
     }
+    auto flush = [&]() {
+#pragma unroll
+        for (int k = 0; k < M; ++k) {
+            U[k] += lg2(PU[k]);
+            V[k] += lg2(PV[k]);
+            PU[k] = 1.f;
+            PV[k] = 1.f;
+        }
+    };
     // column pairs (j, j+1) as packed fp32x2 values
     constexpr int M2 = M / 2;
     float2 E2[M][M2];
     auto anchor = [&]() {
+        flush();
 #pragma unroll
         for (int i = 0; i < M; ++i)
 #pragma unroll
             for (int v = 0; v < M / 4; ++v) {
                 const float4 q = lds4_keep(y0s + i * M + 4 * v);
-                const float u = float(U[i]);
-                const float2 a = add2(make_float2(q.x, q.y), add2(make_float2(u, u), make_float2(float(V[4 * v]), float(V[4 * v + 1]))));
-                const float2 c = add2(make_float2(q.z, q.w), add2(make_float2(u, u), make_float2(float(V[4 * v + 2]), float(V[4 * v + 3]))));
+                const float2 u2 = make_float2(U[i], U[i]);
+                const float2 a = add2(make_float2(q.x, q.y), add2(u2, make_float2(V[4 * v], V[4 * v + 1])));
+                const float2 c = add2(make_float2(q.z, q.w), add2(u2, make_float2(V[4 * v + 2], V[4 * v + 3])));
                 E2[i][2 * v] = make_float2(ex2(a.x), ex2(a.y));
                 E2[i][2 * v + 1] = make_float2(ex2(c.x), ex2(c.y));
             }
@@ -163,26 +179,28 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
                 float2 acc = e2[0];
 #pragma unroll
                 for (int c = 1; c < M2; ++c) acc = add2(acc, e2[c]);
-                const float r = log2N - lg2(acc.x + acc.y);
-                const float w = ex2(r);                  // N / R_i
+                const float w = fN * rcp(acc.x + acc.y);   // N / R_i = 2^r_i
                 const float2 w2 = make_float2(w, w);
 #pragma unroll
                 for (int c = 0; c < M2; ++c) {
                     C2[c] = fma2(e2[c], w2, C2[c]);
                     E2[i][c] = mul2(E2[i][c], w2);
                 }
-                U[i] += Acc(r);
-                if constexpr (EXT) delta = fmaxf(delta, fabsf(r));
+                PU[i] *= w;
+                if constexpr (EXT) {
+                    if (ext.tol2 > 0.f) delta = fmaxf(delta, fabsf(lg2(w)));
+                }
             }
 #pragma unroll
             for (int c = 0; c < M2; ++c) {
-                const float2 cv = make_float2(log2N - lg2(C2[c].x), log2N - lg2(C2[c].y));
-                const float2 u2 = make_float2(ex2(cv.x), ex2(cv.y));   // N / C_j
+                const float2 u2 = make_float2(fN * rcp(C2[c].x), fN * rcp(C2[c].y));   // N / C_j = 2^c_j
 #pragma unroll
                 for (int i = 0; i < M; ++i) E2[i][c] = mul2(E2[i][c], u2);
-                V[2 * c] += Acc(cv.x);
-                V[2 * c + 1] += Acc(cv.y);
-                if constexpr (EXT) delta = fmaxf(delta, fmaxf(fabsf(cv.x), fabsf(cv.y)));
+                PV[2 * c] *= u2.x;
+                PV[2 * c + 1] *= u2.y;
+                if constexpr (EXT) {
+                    if (ext.tol2 > 0.f) delta = fmaxf(delta, fmaxf(fabsf(lg2(u2.x)), fabsf(lg2(u2.y))));
+                }
             }
             used = t + 1;
             if constexpr (EXT) {
@@ -199,11 +217,12 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
         }
     if constexpr (EXT) {
         if (ext.potentials) {
+            flush();
             float* uv = ext.potentials + 2 * M * b;
 #pragma unroll
             for (int k = 0; k < M; ++k) {
-                uv[k] = finite ? float(U[k] * kLn2D) : __int_as_float(0x7fc00000);
-                uv[M + k] = finite ? float(V[k] * kLn2D) : __int_as_float(0x7fc00000);
+                uv[k] = finite ? float(double(U[k]) * kLn2D) : __int_as_float(0x7fc00000);
+                uv[M + k] = finite ? float(double(V[k]) * kLn2D) : __int_as_float(0x7fc00000);
             }
         }
         if (ext.iters_used) ext.iters_used[b] = finite ? used : 0;
@@ -325,11 +344,12 @@ struct TileSource {
 // are the whole state.  The clipped exponentials e = 2^min(y, 0) are not
 // taken afresh every iteration: E = 2^y is carried from one iteration to the
 // next by the same update in linear form, E <- E * 2^r_i * 2^c_j (the
-// exponential of y += r_i + c_j, with r_i = log2 N - log2 R_i and
-// c_j = log2 N - log2 C_j, the very values summed into U and V), and
-// re-anchored to 2^(y0 + U + V) every kAnchorEvery iterations, so that an
-// entry that underflowed for a while recovers and the rounding of the
-// products never builds up.
+// exponential of y += r_i + c_j, with 2^r_i = N / R_i and 2^c_j = N / C_j by
+// the hardware reciprocal).  The owners keep the products of the factors
+// they applied since the last anchor point; every kAnchorEvery iterations
+// their base-2 logarithms are added to U and V and E is re-anchored to
+// 2^(y0 + U + V), so that an entry that underflowed for a while recovers and
+// the rounding of the products never builds up.
 
 // EXT: warm start from / export to ext.potentials of block b, stop rule
 // ext.tol2, iteration count to ext.iters_used.
@@ -452,11 +472,24 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
             const float q1 = m > 0.f ? __fdiv_rn(y[k][2 * c + 1], m) : 0.f;
             y0t[(k * Q2 + c) * C::TPB] = make_float2(fmaf(tau2, q0, -tau2), fmaf(tau2, q1, -tau2));
         }
-    const float log2N = log2f(float(N));
+    const float fN = float(N);
 
     // potentials of the owned rows (register k < RO holds row(k)) and columns
-    // (c < CO holds col(c)); EXT may start them from ext.potentials (nats)
+    // (c < CO holds col(c)) as of the last anchor point (EXT may start them
+    // from ext.potentials, nats), and the products of the scalings applied
+    // since then, whose base-2 logarithms are added at the next anchor point
     double ua[C::RO], va[C::CO];
+    float pu[C::RO], pv[C::CO];
+#pragma unroll
+    for (int lo = 0; lo < C::RO; ++lo) pu[lo] = 1.f;
+#pragma unroll
+    for (int lo = 0; lo < C::CO; ++lo) pv[lo] = 1.f;
+    auto flush = [&]() {
+#pragma unroll
+        for (int lo = 0; lo < C::RO; ++lo) { ua[lo] += double(lg2(pu[lo])); pu[lo] = 1.f; }
+#pragma unroll
+        for (int lo = 0; lo < C::CO; ++lo) { va[lo] += double(lg2(pv[lo])); pv[lo] = 1.f; }
+    };
     {
         const float* uv = nullptr;
         if constexpr (EXT) uv = (ext.warm && active) ? ext.potentials + 2 * M * b : nullptr;
@@ -470,6 +503,7 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
     // register order)
     float2 E2[P][Q2];                                // 2^y, column pairs packed
     auto anchor = [&]() {
+        flush();
         float U[P], V[Q];
 #pragma unroll
         for (int lo = 0; lo < C::RO; ++lo) U[lo] = float(ua[lo]);
@@ -535,13 +569,10 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
 #pragma unroll
                 for (int lo = 0; lo < C::RO; ++lo)
                     rs[lo] += __shfl_xor_sync(kFullMask, rs[lo], s);
-            // owned rows: log potential r = log2 N - log2 R and scale w = 2^r
-            float wv[P], rv[C::RO];
+            // owned rows: scale w = N / R = 2^r
+            float wv[P];
 #pragma unroll
-            for (int lo = 0; lo < C::RO; ++lo) {
-                rv[lo] = log2N - lg2(rs[lo]);
-                wv[lo] = ex2(rv[lo]);                // N / R_i, consistent with the potential
-            }
+            for (int lo = 0; lo < C::RO; ++lo) wv[lo] = fN * rcp(rs[lo]);
             // all-gather of the scales back into the permuted register order
 #pragma unroll
             for (int s = 1; s < C::RSR; s <<= 1)
@@ -580,13 +611,10 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
                     cs[lo] = acc;
                 }
             }
-            // owned columns: log potential c = log2 N - log2 C and scale u = 2^c
-            float uv[Q], cv[C::CO];
+            // owned columns: scale u = N / C = 2^c
+            float uv[Q];
 #pragma unroll
-            for (int lo = 0; lo < C::CO; ++lo) {
-                cv[lo] = log2N - lg2(cs[lo]);
-                uv[lo] = ex2(cv[lo]);                // N / C_j
-            }
+            for (int lo = 0; lo < C::CO; ++lo) uv[lo] = fN * rcp(cs[lo]);
 #pragma unroll
             for (int s = 1; s < C::RSC; s <<= 1)
 #pragma unroll
@@ -594,7 +622,14 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
 #pragma unroll
                     for (int lo = 0; lo < C::CO; ++lo)
                         uv[(hi + s) * C::CO + lo] = __shfl_xor_sync(kFullMask, uv[hi * C::CO + lo], s * C::CG);
+            float delta = 0.f;                       // EXT: largest |r_i|, |c_j| of the owned ones
             if constexpr (EXT) {
+                if (ext.tol2 > 0.f) {
+#pragma unroll
+                    for (int lo = 0; lo < C::RO; ++lo) delta = fmaxf(delta, fabsf(lg2(wv[lo])));
+#pragma unroll
+                    for (int lo = 0; lo < C::CO; ++lo) delta = fmaxf(delta, fabsf(lg2(uv[lo])));
+                }
                 // a stopped block of a shared warp (M = 16) keeps its state
                 if (done) {
 #pragma unroll
@@ -609,23 +644,11 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
 #pragma unroll
                 for (int c = 0; c < Q2; ++c)
                     E2[k][c] = mul2(E2[k][c], mul2(make_float2(wv[k], wv[k]), make_float2(uv[2 * c], uv[2 * c + 1])));
-            if constexpr (!EXT) {
 #pragma unroll
-                for (int lo = 0; lo < C::RO; ++lo) ua[lo] += double(rv[lo]);
+            for (int lo = 0; lo < C::RO; ++lo) pu[lo] *= wv[lo];
 #pragma unroll
-                for (int lo = 0; lo < C::CO; ++lo) va[lo] += double(cv[lo]);
-            } else {
-                float delta = 0.f;
-#pragma unroll
-                for (int lo = 0; lo < C::RO; ++lo) {
-                    if (!done) ua[lo] += double(rv[lo]);
-                    delta = fmaxf(delta, fabsf(rv[lo]));
-                }
-#pragma unroll
-                for (int lo = 0; lo < C::CO; ++lo) {
-                    if (!done) va[lo] += double(cv[lo]);
-                    delta = fmaxf(delta, fabsf(cv[lo]));
-                }
+            for (int lo = 0; lo < C::CO; ++lo) pv[lo] *= uv[lo];
+            if constexpr (EXT) {
                 if (!done) used = it + 1;
                 if (ext.tol2 > 0.f) {
                     const bool small = delta <= ext.tol2;
@@ -654,6 +677,7 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
             y[k][2 * c + 1] = fminf(E2[k][c].y, 1.f);
         }
     if constexpr (EXT) {
+        flush();
         if (active) {
             if (ext.potentials) {
                 float* uv = ext.potentials + 2 * M * b;
