@@ -46,6 +46,11 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d.u) : "l"(x.u), "l"(y.u));
     return d.f;
 }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    F2U x{a}, y{b}, d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d.u) : "l"(x.u), "l"(y.u));
+    return d.f;
+}
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
     F2U x{a}, y{b}, d;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.u) : "l"(x.u), "l"(y.u));

@@ -101,6 +101,7 @@ struct RoundView {
     int* bestp;                         // ... and that partner (lowest index on ties)
     int* rc;                            // row counts (greedy, repair)
     int* cc;                            // column counts
+    float* sc;                          // M <= 32: 4*M floats, 16-byte aligned (local search)
 };
 
 // Per-block shared memory of the rounding steps after the sort (M <= 32).
@@ -120,7 +121,8 @@ struct RoundShared {
     int bestp[M];
     int rc[M];
     int cc[M];
-    __device__ __forceinline__ RoundView<M> view() { return RoundView<M>{G, order, rowbits, bestv, bestp, rc, cc}; }
+    float sc[4 * M];                    // local search: C and Bn of the two rows of the last swap
+    __device__ __forceinline__ RoundView<M> view() { return RoundView<M>{G, order, rowbits, bestv, bestp, rc, cc, sc}; }
 };
 
 // Bitonic compare-exchange of registers r and r|J of this lane: the pair ends
@@ -351,6 +353,13 @@ __device__ bool greedy_and_repair(const float* a, const RoundView<M>& sh, int N,
 // of 4 warps for M = 64); thread tid serves partner row y = tid / CH and
 // columns [h*CPT, (h+1)*CPT) of it, h = tid % CH.  Each thread keeps those
 // |W| values of its row in registers.
+// 3-input maximum (sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 template <int M>
 struct LsCfg {
     static constexpr int NT = M <= 32 ? 32 : 128;
@@ -437,6 +446,26 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
     }
     ls_barrier<NT>();
     if (row_thread && h == 0) rescan_row<M>(sh, y);
+
+    // The sweeps compute pair gains in max-plus form: with C_x[j] = a_xj off
+    // row x's support (-inf on it) and Bn_x[j] = a_xj on it (+inf off it),
+    // max over j in O_x \ O_y of (a_yj - a_xj) = max_j (C_y[j] - Bn_x[j]) and
+    // max over j in O_y \ O_x of (a_xj - a_yj) = max_j (C_x[j] - Bn_y[j]):
+    // the same fp32 differences, with no per-column tests.  Each lane keeps
+    // its own row in that form; after a swap the two changed rows are written
+    // to sh.sc, where every lane reads them.
+    static_assert(NT == 32 && CH == 1 && M % 4 == 0, "one row per lane");
+    constexpr int M2 = M / 2;
+    float2 Cy[M2], Bny[M2];
+    {
+        const Bits Oy = row_thread ? sh.rowbits[y] : Bits(0);
+#pragma unroll
+        for (int c = 0; c < M2; ++c) {
+            const bool in0 = (Oy >> (2 * c)) & 1, in1 = (Oy >> (2 * c + 1)) & 1;
+            Cy[c] = make_float2(in0 ? -INFINITY : ay[2 * c], in1 ? -INFINITY : ay[2 * c + 1]);
+            Bny[c] = make_float2(in0 ? ay[2 * c] : INFINITY, in1 ? ay[2 * c + 1] : INFINITY);
+        }
+    }
     ls_barrier<NT>();
 
     int quiet = 0;                                   // anchors in a row without a swap
@@ -455,19 +484,14 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
             const int bp = sh.bestp[i];
             if (!(best > 0.f)) { ++quiet; continue; }
             const Bits Oi = sh.rowbits[i], Ob = sh.rowbits[bp];
-            // entries to exchange (every warp finds the same pair): lowest index on ties
+            // entries to exchange (every lane finds the same pair): lowest index on ties
             float v1 = -INFINITY, v2 = -INFINITY;
             int j1 = INT_MAX, j2 = INT_MAX;
-            for (int jj = lane; jj < M; jj += 32) {
-                const bool in_i = (Oi >> jj) & 1, in_p = (Ob >> jj) & 1;
-                if (in_i && !in_p) {
-                    const float d = __fsub_rn(a[bp * AS + jj], a[i * AS + jj]);
-                    if (j1 == INT_MAX || d > v1) { v1 = d; j1 = jj; }
-                }
-                if (!in_i && in_p) {
-                    const float d = __fsub_rn(a[i * AS + jj], a[bp * AS + jj]);
-                    if (j2 == INT_MAX || d > v2) { v2 = d; j2 = jj; }
-                }
+            const float ai = row_thread ? a[i * AS + lane] : 0.f, ab = row_thread ? a[bp * AS + lane] : 0.f;
+            if (row_thread) {
+                const bool in_i = (Oi >> lane) & 1, in_p = (Ob >> lane) & 1;
+                if (in_i && !in_p) { v1 = __fsub_rn(ab, ai); j1 = lane; }
+                if (!in_i && in_p) { v2 = __fsub_rn(ai, ab); j2 = lane; }
             }
             warp_argmax(v1, j1);
             warp_argmax(v2, j2);
@@ -475,27 +499,58 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
             quiet = 0;
             const Bits Oi2 = (Oi & ~(Bits(1) << j1)) | (Bits(1) << j2);
             const Bits Ob2 = (Ob & ~(Bits(1) << j2)) | (Bits(1) << j1);
-            const Bits Oy = !row_thread ? Bits(0) : (y == i) ? Oi2 : (y == bp) ? Ob2 : sh.rowbits[y];
             ls_barrier<NT>();                        // everyone has read the old rows
             if (tid == 0) {
                 sh.rowbits[i] = Oi2;
                 sh.rowbits[bp] = Ob2;
             }
-            // new gains g(i, y) and g(bp, y) of partner row y
-            float t1i = -INFINITY, t2i = -INFINITY, t1b = -INFINITY, t2b = -INFINITY;
-            if (row_thread) {
-                pair_pieces<M, CPT, Bits>(ay, a + i * AS, Oi2, Oy, j0, t1i, t2i);
-                pair_pieces<M, CPT, Bits>(ay, a + bp * AS, Ob2, Oy, j0, t1b, t2b);
+            if (row_thread) {                        // rows i and bp after the swap: C, Bn, C, Bn
+                const bool ni = (Oi2 >> lane) & 1, nb = (Ob2 >> lane) & 1;
+                sh.sc[lane] = ni ? -INFINITY : ai;
+                sh.sc[M + lane] = ni ? ai : INFINITY;
+                sh.sc[2 * M + lane] = nb ? -INFINITY : ab;
+                sh.sc[3 * M + lane] = nb ? ab : INFINITY;
             }
-            t1i = row_max<CH>(t1i); t2i = row_max<CH>(t2i);
-            t1b = row_max<CH>(t1b); t2b = row_max<CH>(t2b);
-            const float gi = __fadd_rn(t1i, t2i), gb = __fadd_rn(t1b, t2b);
-            if (row_thread && h == 0) {
+            ls_barrier<NT>();
+            if (y == i || y == bp) {                 // this lane's own row changed
+                const float* src = sh.sc + (y == i ? 0 : 2 * M);
+#pragma unroll
+                for (int q = 0; q < M / 4; ++q) {
+                    const float4 c4 = *reinterpret_cast<const float4*>(src + 4 * q);
+                    const float4 b4 = *reinterpret_cast<const float4*>(src + M + 4 * q);
+                    Cy[2 * q] = make_float2(c4.x, c4.y);
+                    Cy[2 * q + 1] = make_float2(c4.z, c4.w);
+                    Bny[2 * q] = make_float2(b4.x, b4.y);
+                    Bny[2 * q + 1] = make_float2(b4.z, b4.w);
+                }
+            }
+            // new gains g(i, y) and g(bp, y) of partner row y
+            float t1i0 = -INFINITY, t1i1 = -INFINITY, t2i0 = -INFINITY, t2i1 = -INFINITY;
+            float t1b0 = -INFINITY, t1b1 = -INFINITY, t2b0 = -INFINITY, t2b1 = -INFINITY;
+#pragma unroll
+            for (int q = 0; q < M / 4; ++q) {
+                const float4 ci = *reinterpret_cast<const float4*>(sh.sc + 4 * q);
+                const float4 bi = *reinterpret_cast<const float4*>(sh.sc + M + 4 * q);
+                const float4 cb = *reinterpret_cast<const float4*>(sh.sc + 2 * M + 4 * q);
+                const float4 bb = *reinterpret_cast<const float4*>(sh.sc + 3 * M + 4 * q);
+                float2 d;
+                d = sub2(Cy[2 * q], make_float2(bi.x, bi.y));     t1i0 = max3f(t1i0, d.x, d.y);
+                d = sub2(Cy[2 * q + 1], make_float2(bi.z, bi.w)); t1i1 = max3f(t1i1, d.x, d.y);
+                d = sub2(make_float2(ci.x, ci.y), Bny[2 * q]);     t2i0 = max3f(t2i0, d.x, d.y);
+                d = sub2(make_float2(ci.z, ci.w), Bny[2 * q + 1]); t2i1 = max3f(t2i1, d.x, d.y);
+                d = sub2(Cy[2 * q], make_float2(bb.x, bb.y));     t1b0 = max3f(t1b0, d.x, d.y);
+                d = sub2(Cy[2 * q + 1], make_float2(bb.z, bb.w)); t1b1 = max3f(t1b1, d.x, d.y);
+                d = sub2(make_float2(cb.x, cb.y), Bny[2 * q]);     t2b0 = max3f(t2b0, d.x, d.y);
+                d = sub2(make_float2(cb.z, cb.w), Bny[2 * q + 1]); t2b1 = max3f(t2b1, d.x, d.y);
+            }
+            const float gi = __fadd_rn(fmaxf(t1i0, t1i1), fmaxf(t2i0, t2i1));
+            const float gb = __fadd_rn(fmaxf(t1b0, t1b1), fmaxf(t2b0, t2b1));
+            if (row_thread) {
                 if (y != i) { sh.G[i * GS + y] = gi; sh.G[y * GS + i] = gi; }
                 if (y != i && y != bp) { sh.G[bp * GS + y] = gb; sh.G[y * GS + bp] = gb; }
             }
             ls_barrier<NT>();                        // gain table and rows complete
-            if (row_thread && h == 0) {
+            if (row_thread) {
                 const int op = sh.bestp[y];
                 if (y == i || y == bp || op == i || op == bp) {
                     rescan_row<M>(sh, y);
@@ -620,12 +675,6 @@ constexpr size_t round_warp_smem() { return sizeof(RoundWarpSmem<M>) * 4; }
 // bit-tested form used for M <= 32, with no per-column tests.
 // ---------------------------------------------------------------------------
 
-// 3-input maximum (sm_100).
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
 
 // B and C rows in shared memory (row stride M floats) keep their 16-byte
 // chunks XOR-swizzled by the row index, so that threads reading chunk c of
@@ -836,7 +885,7 @@ struct Round64Smem {
     int ok;
     uint64_t tma_bar;                                // fused kernel: completion of the W tile copy
     __device__ __forceinline__ RoundView<64> view() {
-        return RoundView<64>{a, u.gr.order, v.rb.rowbits, v.rb.bestv, v.rb.bestp, u.gr.rc, u.gr.cc};
+        return RoundView<64>{a, u.gr.order, v.rb.rowbits, v.rb.bestv, v.rb.bestp, u.gr.rc, u.gr.cc, nullptr};
     }
 };
 
