@@ -66,13 +66,12 @@ __device__ __forceinline__ float4 lds4_keep(const float* p) {
 }
 
 // Dykstra for block b (rows r0.., columns c0..) by one thread, in the form of
-// dykstra_tile_solve: the state is y = y0 + U_i + V_j, E = 2^y is carried in
-// linear form between anchor points (E *= 2^r_i after row i's step,
-// E *= 2^c_j after the column step) and recomputed from y0 + U + V every
-// kAnchorEvery iterations.  The scalings are N / R_i and N / C_j by the
-// hardware reciprocal; their products since the last anchor point are kept
-// per row and column and their base-2 logarithms added to U and V (fp32) at
-// the next one, so the potentials follow the very factors applied to E.
+// dykstra_tile_solve: the state is y = y0 + U_i + V_j, E = 2^y = F / TH_i is
+// carried in linear form between anchor points (the row step sets the row's
+// clip threshold TH_i, the column step multiplies F by N / C_j) and
+// recomputed from y0 + U + V every kAnchorEvery iterations, when the
+// logarithms of the thresholds and of the column factors' products are added
+// to U and V (fp32), so the potentials follow the very factors applied.
 // y0s: this thread's M*M floats of shared memory (16-byte aligned), which
 // hold y0 during the iterations.  On return `s` holds the plan
 // 2^min(y, 0); returns whether the block's W is finite.
@@ -117,10 +116,12 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
     }
     const float fN = float(N);
 
-    // potentials (log2 units) as of the last anchor point, and the products of
-    // the row and column scalings applied since then (their logarithms are
-    // added at the next anchor point)
-    float U[M], V[M], PU[M], PV[M];
+    // potentials (log2 units) as of the last anchor point; since then each
+    // row's scaling lives in its clip threshold TH (E = F / TH, see
+    // dykstra_tile_solve) and the column scalings multiply F, their products
+    // kept in PV; both are added to U and V at the next anchor point
+    const float invN = 1.f / float(N);
+    float U[M], V[M], TH[M], PV[M];
     int used = 0;
     {
         const float* uv = nullptr;
@@ -129,24 +130,25 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
         for (int k = 0; k < M; ++k) {
             U[k] = uv ? float(double(uv[k]) * kLog2eD) : 0.f;
             V[k] = uv ? float(double(uv[M + k]) * kLog2eD) : 0.f;
-            PU[k] = 1.f;
+            TH[k] = 1.f;
             PV[k] = 1.f;
         }
     }
     auto flush = [&]() {
 #pragma unroll
         for (int k = 0; k < M; ++k) {
-            U[k] += lg2(PU[k]);
+            U[k] -= lg2(TH[k]);
             V[k] += lg2(PV[k]);
-            PU[k] = 1.f;
             PV[k] = 1.f;
         }
     };
     // column pairs (j, j+1) as packed fp32x2 values
     constexpr int M2 = M / 2;
-    float2 E2[M][M2];
+    float2 E2[M][M2];                                // F
     auto anchor = [&]() {
         flush();
+#pragma unroll
+        for (int k = 0; k < M; ++k) TH[k] = 1.f;
 #pragma unroll
         for (int i = 0; i < M; ++i)
 #pragma unroll
@@ -175,21 +177,20 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
             for (int i = 0; i < M; ++i) {
                 float2 e2[M2];
 #pragma unroll
-                for (int c = 0; c < M2; ++c) e2[c] = make_float2(fminf(E2[i][c].x, 1.f), fminf(E2[i][c].y, 1.f));
+                for (int c = 0; c < M2; ++c) e2[c] = make_float2(fminf(E2[i][c].x, TH[i]), fminf(E2[i][c].y, TH[i]));
                 float2 acc = e2[0];
 #pragma unroll
                 for (int c = 1; c < M2; ++c) acc = add2(acc, e2[c]);
-                const float w = fN * rcp(acc.x + acc.y);   // N / R_i = 2^r_i
+                const float S = acc.x + acc.y;
+                const float w = fN * rcp(S);             // weight of min(F, TH) in the column step
                 const float2 w2 = make_float2(w, w);
 #pragma unroll
-                for (int c = 0; c < M2; ++c) {
-                    C2[c] = fma2(e2[c], w2, C2[c]);
-                    E2[i][c] = mul2(E2[i][c], w2);
-                }
-                PU[i] *= w;
+                for (int c = 0; c < M2; ++c) C2[c] = fma2(e2[c], w2, C2[c]);
+                const float tn = S * invN;               // threshold after the row step
                 if constexpr (EXT) {
-                    if (ext.tol2 > 0.f) delta = fmaxf(delta, fabsf(lg2(w)));
+                    if (ext.tol2 > 0.f) delta = fmaxf(delta, fabsf(lg2(TH[i]) - lg2(tn)));
                 }
+                TH[i] = tn;
             }
 #pragma unroll
             for (int c = 0; c < M2; ++c) {
@@ -209,12 +210,14 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
         }
     }
 #pragma unroll
-    for (int i = 0; i < M; ++i)
+    for (int i = 0; i < M; ++i) {
+        const float rho = rcp(TH[i]);
 #pragma unroll
         for (int c = 0; c < M2; ++c) {
-            y[i][2 * c] = fminf(E2[i][c].x, 1.f);
-            y[i][2 * c + 1] = fminf(E2[i][c].y, 1.f);
+            y[i][2 * c] = fminf(E2[i][c].x * rho, 1.f);
+            y[i][2 * c + 1] = fminf(E2[i][c].y * rho, 1.f);
         }
+    }
     if constexpr (EXT) {
         if (ext.potentials) {
             flush();
@@ -344,12 +347,16 @@ struct TileSource {
 // are the whole state.  The clipped exponentials e = 2^min(y, 0) are not
 // taken afresh every iteration: E = 2^y is carried from one iteration to the
 // next by the same update in linear form, E <- E * 2^r_i * 2^c_j (the
-// exponential of y += r_i + c_j, with 2^r_i = N / R_i and 2^c_j = N / C_j by
-// the hardware reciprocal).  The owners keep the products of the factors
-// they applied since the last anchor point; every kAnchorEvery iterations
-// their base-2 logarithms are added to U and V and E is re-anchored to
-// 2^(y0 + U + V), so that an entry that underflowed for a while recovers and
-// the rounding of the products never builds up.
+// exponential of y += r_i + c_j, 2^r_i = N / R_i and 2^c_j = N / C_j).  The
+// row factor is not applied entry by entry: E_ij = F_ij / th_i, the clip
+// min(E, 1) = min(F, th_i) / th_i, and the row step replaces th_i by S_i / N
+// (S_i = sum_j min(F_ij, th_i)), which is the same as multiplying row i of E
+// by N / R_i; the column step multiplies F by N / C_j (hardware reciprocal),
+// so one multiply per entry and iteration remains.  Every kAnchorEvery
+// iterations log2 of the threshold and of the column factors' product are
+// added to U and V, and E is re-anchored to 2^(y0 + U + V) (th = 1), so that
+// an entry that underflowed for a while recovers and the rounding of the
+// products never builds up.
 
 // EXT: warm start from / export to ext.potentials of block b, stop rule
 // ext.tol2, iteration count to ext.iters_used.
@@ -476,17 +483,22 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
 
     // potentials of the owned rows (register k < RO holds row(k)) and columns
     // (c < CO holds col(c)) as of the last anchor point (EXT may start them
-    // from ext.potentials, nats), and the products of the scalings applied
-    // since then, whose base-2 logarithms are added at the next anchor point
+    // from ext.potentials, nats).  Since then: each row's scaling lives in
+    // its clip threshold thr[k] (E_ij = F_ij / th_i, so min(E, 1) is
+    // min(F, th_i) / th_i and the row step sets th_i = S_i / N with
+    // S_i = sum_j min(F_ij, th_i)), which makes the row's potential step
+    // log2(th_old / th_new); the column scalings multiply F, and the owners
+    // keep their products.  Both are added to U and V at the next anchor point.
+    const float invN = 1.f / float(N);
     double ua[C::RO], va[C::CO];
-    float pu[C::RO], pv[C::CO];
+    float thr[P], pv[C::CO];
 #pragma unroll
-    for (int lo = 0; lo < C::RO; ++lo) pu[lo] = 1.f;
+    for (int k = 0; k < P; ++k) thr[k] = 1.f;
 #pragma unroll
     for (int lo = 0; lo < C::CO; ++lo) pv[lo] = 1.f;
     auto flush = [&]() {
 #pragma unroll
-        for (int lo = 0; lo < C::RO; ++lo) { ua[lo] += double(lg2(pu[lo])); pu[lo] = 1.f; }
+        for (int lo = 0; lo < C::RO; ++lo) ua[lo] -= double(lg2(thr[lo]));
 #pragma unroll
         for (int lo = 0; lo < C::CO; ++lo) { va[lo] += double(lg2(pv[lo])); pv[lo] = 1.f; }
     };
@@ -498,12 +510,14 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
 #pragma unroll
         for (int lo = 0; lo < C::CO; ++lo) va[lo] = uv ? double(uv[M + th.col(lo)]) * kLog2eD : 0.0;
     }
-    // E = 2^(y0 + U_i + V_j) over this thread's entries (the potentials,
-    // rounded to fp32, all-gathered from their owners into the permuted
-    // register order)
-    float2 E2[P][Q2];                                // 2^y, column pairs packed
+    // F = E = 2^(y0 + U_i + V_j) over this thread's entries and th = 1 (the
+    // potentials, rounded to fp32, all-gathered from their owners into the
+    // permuted register order)
+    float2 F2[P][Q2];                                // column pairs packed
     auto anchor = [&]() {
         flush();
+#pragma unroll
+        for (int k = 0; k < P; ++k) thr[k] = 1.f;
         float U[P], V[Q];
 #pragma unroll
         for (int lo = 0; lo < C::RO; ++lo) U[lo] = float(ua[lo]);
@@ -529,7 +543,7 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
             for (int c = 0; c < Q2; ++c) {
                 const float2 uv2 = add2(make_float2(U[k], U[k]), make_float2(V[2 * c], V[2 * c + 1]));
                 const float2 y2 = add2(lds_keep(y0t + (k * Q2 + c) * C::TPB), uv2);
-                E2[k][c] = make_float2(ex2(y2.x), ex2(y2.y));
+                F2[k][c] = make_float2(ex2(y2.x), ex2(y2.y));
             }
     };
     anchor();
@@ -552,7 +566,7 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
 #pragma unroll
             for (int k = 0; k < P; ++k) {
 #pragma unroll
-                for (int c = 0; c < Q2; ++c) e2[k][c] = make_float2(fminf(E2[k][c].x, 1.f), fminf(E2[k][c].y, 1.f));
+                for (int c = 0; c < Q2; ++c) e2[k][c] = make_float2(fminf(F2[k][c].x, thr[k]), fminf(F2[k][c].y, thr[k]));
                 const float2 acc = add2(add2(e2[k][0], e2[k][1]), add2(e2[k][2], e2[k][3]));
                 rs[k] = acc.x + acc.y;
             }
@@ -569,10 +583,14 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
 #pragma unroll
                 for (int lo = 0; lo < C::RO; ++lo)
                     rs[lo] += __shfl_xor_sync(kFullMask, rs[lo], s);
-            // owned rows: scale w = N / R = 2^r
-            float wv[P];
+            // owned rows: column-step weight N / S (= e's scale N / R over th) and
+            // the next threshold S / N
+            float wv[P], tn[P];
 #pragma unroll
-            for (int lo = 0; lo < C::RO; ++lo) wv[lo] = fN * rcp(rs[lo]);
+            for (int lo = 0; lo < C::RO; ++lo) {
+                wv[lo] = fN * rcp(rs[lo]);
+                tn[lo] = rs[lo] * invN;
+            }
             // all-gather of the scales back into the permuted register order
 #pragma unroll
             for (int s = 1; s < C::RSR; s <<= 1)
@@ -580,7 +598,10 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
                 for (int hi = 0; hi < s; ++hi)
 #pragma unroll
                     for (int lo = 0; lo < C::RO; ++lo)
+                    {
                         wv[(hi + s) * C::RO + lo] = __shfl_xor_sync(kFullMask, wv[hi * C::RO + lo], s);
+                        tn[(hi + s) * C::RO + lo] = __shfl_xor_sync(kFullMask, tn[hi * C::RO + lo], s);
+                    }
             // column partial sums of e * w
             float cs[Q];
 #pragma unroll
@@ -626,26 +647,25 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
             if constexpr (EXT) {
                 if (ext.tol2 > 0.f) {
 #pragma unroll
-                    for (int lo = 0; lo < C::RO; ++lo) delta = fmaxf(delta, fabsf(lg2(wv[lo])));
+                    for (int lo = 0; lo < C::RO; ++lo) delta = fmaxf(delta, fabsf(lg2(thr[lo]) - lg2(tn[lo])));
 #pragma unroll
                     for (int lo = 0; lo < C::CO; ++lo) delta = fmaxf(delta, fabsf(lg2(uv[lo])));
                 }
                 // a stopped block of a shared warp (M = 16) keeps its state
                 if (done) {
 #pragma unroll
-                    for (int k = 0; k < P; ++k) wv[k] = 1.f;
+                    for (int k = 0; k < P; ++k) tn[k] = thr[k];
 #pragma unroll
                     for (int c = 0; c < Q; ++c) uv[c] = 1.f;
                 }
             }
-            // y += r_i + c_j, in both forms
+            // y += r_i + c_j: the row part through the thresholds, the column part on F
 #pragma unroll
-            for (int k = 0; k < P; ++k)
+            for (int k = 0; k < P; ++k) {
+                thr[k] = tn[k];
 #pragma unroll
-                for (int c = 0; c < Q2; ++c)
-                    E2[k][c] = mul2(E2[k][c], mul2(make_float2(wv[k], wv[k]), make_float2(uv[2 * c], uv[2 * c + 1])));
-#pragma unroll
-            for (int lo = 0; lo < C::RO; ++lo) pu[lo] *= wv[lo];
+                for (int c = 0; c < Q2; ++c) F2[k][c] = mul2(F2[k][c], make_float2(uv[2 * c], uv[2 * c + 1]));
+            }
 #pragma unroll
             for (int lo = 0; lo < C::CO; ++lo) pv[lo] *= uv[lo];
             if constexpr (EXT) {
@@ -673,8 +693,9 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
     for (int k = 0; k < P; ++k)
 #pragma unroll
         for (int c = 0; c < Q2; ++c) {
-            y[k][2 * c] = fminf(E2[k][c].x, 1.f);
-            y[k][2 * c + 1] = fminf(E2[k][c].y, 1.f);
+            const float rho = rcp(thr[k]);
+            y[k][2 * c] = fminf(F2[k][c].x * rho, 1.f);
+            y[k][2 * c + 1] = fminf(F2[k][c].y * rho, 1.f);
         }
     if constexpr (EXT) {
         flush();
