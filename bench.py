@@ -37,9 +37,10 @@ STACK = "stack7b"                  # 32 layers x 7 matrices, 4:8, one pass = one
 SM_COUNT = 148
 FP32_LANES_PER_CLK_PER_SM = 128   # fp32 add / mul / fma results per clock per SM (FMA pipe)
 # Algorithmic FMA-pipe work of one Dykstra iteration per entry: the row-sum
-# add, the column-sum fma and the row and column scalings of E (the clip
-# min(E, 1) runs on the ALU pipe and is not counted).
-FP32_OPS_PER_ENTRY_ITER = 4
+# add, the column-sum fma and the column scaling (the row scaling is one
+# threshold per row; the clip min(F, th) runs on the ALU pipe and is not
+# counted).
+FP32_OPS_PER_ENTRY_ITER = 3
 SM_MAX_MHZ_FALLBACK = 1965.0
 L2_FLUSH_BYTES = 256 << 20
 
@@ -678,7 +679,7 @@ def main(argv=None):
         "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TOP/s",
                      "frac": achieved / peak, "traffic": traffic, "kernel": kernel_key,
                      "ops": f"{ops_per_param:.0f} FP32 ops per param = T x {FP32_OPS_PER_ENTRY_ITER} (row-sum add, "
-                            "column-sum fma, row and column scaling of E per entry and iteration)",
+                            "column-sum fma, column scaling per entry and iteration)",
                      "peak_basis": PEAK_BASIS,
                      "kernel_ms": kernel_ms},
         "breakdown_ms": {"dykstra_plan_kernel_alone": plan_ms, "rest_of_step": round_ms,
