@@ -150,6 +150,7 @@ __device__ void group_local_search(const float* a, const RoundView<M>& sh, int s
     for (int jj = 0; jj < M; ++jj) ay[jj] = a[y * AS + jj];
     {
         const Bits Oy = sh.rowbits[y];
+        sh.G[y * GS + y] = -INFINITY;                      // no partner of itself (rescan_row)
 #pragma unroll 1
         for (int d = 1; d <= M / 2; ++d) {
             const int x = (y + d) & (M - 1);

@@ -396,18 +396,28 @@ __device__ __forceinline__ float row_max(float t) {
 }
 
 // Best partner of row x over the cached gains (lowest partner index on ties).
+// The diagonal G[x][x] holds -inf (set with the table), so it never beats a
+// partner: with N < M every row has a partner of finite gain (two rows with
+// the same support in every pair would put M ones in those columns); with
+// N = M every gain is -inf and no swap ever happens, whichever index is kept.
+// Quads are reduced independently, then merged in index order.
 template <int M>
 __device__ __forceinline__ void rescan_row(const RoundView<M>& sh, int x) {
     constexpr int GS = M + 1;
-    float g[M];
-#pragma unroll
-    for (int y = 0; y < M; ++y) g[y] = sh.G[x * GS + y];
+    static_assert(M % 4 == 0, "quads");
+    const float* row = sh.G + x * GS;
     float bv = -INFINITY;
     int bp = -1;
 #pragma unroll
-    for (int y = 0; y < M; ++y) {
-        if (y == x) continue;
-        if (bp < 0 || g[y] > bv) { bv = g[y]; bp = y; }
+    for (int q = 0; q < M / 4; ++q) {
+        const float g0 = row[4 * q], g1 = row[4 * q + 1], g2 = row[4 * q + 2], g3 = row[4 * q + 3];
+        const bool s01 = g1 > g0, s23 = g3 > g2;
+        const float v01 = s01 ? g1 : g0, v23 = s23 ? g3 : g2;
+        const int i01 = 4 * q + (s01 ? 1 : 0), i23 = 4 * q + (s23 ? 3 : 2);
+        const bool s = v23 > v01;
+        const float vq = s ? v23 : v01;
+        const int iq = s ? i23 : i01;
+        if (q == 0 || vq > bv) { bv = vq; bp = iq; }
     }
     sh.bestv[x] = bv;
     sh.bestp[x] = bp;
@@ -430,6 +440,7 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
     // gain table: row y with rows y+1 .. y+M/2 (mod M), every unordered pair once
     {
         const Bits Oy = row_thread ? sh.rowbits[y] : Bits(0);
+        if (row_thread && h == 0) sh.G[y * GS + y] = -INFINITY;   // no partner of itself (rescan_row)
 #pragma unroll 1
         for (int d = 1; d <= M / 2; ++d) {
             const int x = (y + d) & (M - 1);
