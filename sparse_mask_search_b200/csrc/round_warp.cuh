@@ -742,9 +742,11 @@ __device__ __forceinline__ void rescan_row_pair(const RoundView<M>& sh, int x, i
 
 // Step 4 for one M = 64 block by 128 threads.  `a`: |W| (row stride M+1),
 // read only until the B/C arrays are built; sh.G may overlay it.  Bm, Cm:
-// M x M floats each (swizzled rows, bc_index), 16-byte aligned.
+// M x M floats each (swizzled rows, bc_index), 16-byte aligned; xj: two ints
+// of shared memory (the pair of each swap).
 template <int M>
-__device__ void local_search_mp(const float* a, float* Bm, float* Cm, const RoundView<M>& sh, int sweeps, int tid) {
+__device__ void local_search_mp(const float* a, float* Bm, float* Cm, const RoundView<M>& sh, int* xj, int sweeps,
+                                int tid) {
     using L = LsCfg<M>;
     using Bits = typename WarpRound<M>::Bits;
     constexpr int AS = M + 1, GS = M + 1, CH = L::CH, CPT = L::CPT;
@@ -802,37 +804,48 @@ __device__ void local_search_mp(const float* a, float* Bm, float* Cm, const Roun
             const float best = sh.bestv[i];
             const int bp = sh.bestp[i];
             if (!(best > 0.f)) { ++quiet; continue; }
-            // entries to exchange (every warp finds the same pair): lowest index on ties
-            float v1 = -INFINITY, v2 = -INFINITY;
-            int j1 = INT_MAX, j2 = INT_MAX;
+            // entries to exchange, by warp 0 alone (lowest index on ties), which
+            // also applies the swap: since the last barrier no other warp has
+            // read rows i and bp, and the next barrier publishes the result
+            if (tid < 32) {
+                float v1 = -INFINITY, v2 = -INFINITY;
+                int j1 = INT_MAX, j2 = INT_MAX;
 #pragma unroll
-            for (int jj = lane; jj < M; jj += 32) {
-                const int ei = bc_index<M>(i, jj), eb = bc_index<M>(bp, jj);
-                const float d1 = Cm[eb] + Bm[ei];                      // j in O_i \ O_bp: a_bp,j - a_ij
-                if (d1 > -INFINITY && (j1 == INT_MAX || d1 > v1)) { v1 = d1; j1 = jj; }
-                const float d2 = Cm[ei] + Bm[eb];                      // j in O_bp \ O_i: a_ij - a_bp,j
-                if (d2 > -INFINITY && (j2 == INT_MAX || d2 > v2)) { v2 = d2; j2 = jj; }
+                for (int jj = lane; jj < M; jj += 32) {
+                    const int ei = bc_index<M>(i, jj), eb = bc_index<M>(bp, jj);
+                    const float d1 = Cm[eb] + Bm[ei];                  // j in O_i \ O_bp: a_bp,j - a_ij
+                    if (d1 > -INFINITY && (j1 == INT_MAX || d1 > v1)) { v1 = d1; j1 = jj; }
+                    const float d2 = Cm[ei] + Bm[eb];                  // j in O_bp \ O_i: a_ij - a_bp,j
+                    if (d2 > -INFINITY && (j2 == INT_MAX || d2 > v2)) { v2 = d2; j2 = jj; }
+                }
+                warp_argmax(v1, j1);
+                warp_argmax(v2, j2);
+                __syncwarp();                        // the warp has read rows i and bp
+                if (j1 < M && j2 < M) {              // always: a positive gain needs both sets
+                    if (tid < 4) {
+                        // j1 leaves row i for row bp, j2 leaves row bp for row i: one entry per thread
+                        const int r = tid < 2 ? i : bp;
+                        const int j = (tid == 0 || tid == 3) ? j1 : j2;
+                        const int e = bc_index<M>(r, j);
+                        const bool leaves = (tid & 1) == 0;   // (i, j1) and (bp, j2) leave their rows
+                        const float b = Bm[e], c = Cm[e];
+                        Bm[e] = leaves ? -INFINITY : -c;
+                        Cm[e] = leaves ? -b : -INFINITY;
+                    } else if (tid == 4) {
+                        const Bits Oi = sh.rowbits[i], Ob = sh.rowbits[bp];
+                        sh.rowbits[i] = (Oi & ~(Bits(1) << j1)) | (Bits(1) << j2);
+                        sh.rowbits[bp] = (Ob & ~(Bits(1) << j2)) | (Bits(1) << j1);
+                    }
+                }
+                if (tid == 0) { xj[0] = j1; xj[1] = j2; }
             }
-            warp_argmax(v1, j1);
-            warp_argmax(v2, j2);
-            if (j1 >= M || j2 >= M) { ++quiet; continue; }   // unreachable: a positive gain needs both sets
+            __syncthreads();                         // rows i and bp updated, the pair published
+            if (xj[0] >= M || xj[1] >= M) {          // unreachable (uniform)
+                __syncthreads();                     // xj read by all before warp 0 writes it again
+                ++quiet;
+                continue;
+            }
             quiet = 0;
-            const Bits Oi = sh.rowbits[i], Ob = sh.rowbits[bp];
-            __syncthreads();                         // everyone has read rows i and bp
-            if (tid < 4) {
-                // j1 leaves row i for row bp, j2 leaves row bp for row i: one entry per thread
-                const int r = tid < 2 ? i : bp;
-                const int j = (tid == 0 || tid == 3) ? j1 : j2;
-                const int e = bc_index<M>(r, j);
-                const bool leaves = (tid & 1) == 0;  // (i, j1) and (bp, j2) leave their rows
-                const float b = Bm[e], c = Cm[e];
-                Bm[e] = leaves ? -INFINITY : -c;
-                Cm[e] = leaves ? -b : -INFINITY;
-            } else if (tid == 4) {
-                sh.rowbits[i] = (Oi & ~(Bits(1) << j1)) | (Bits(1) << j2);
-                sh.rowbits[bp] = (Ob & ~(Bits(1) << j2)) | (Bits(1) << j1);
-            }
-            __syncthreads();                         // rows i and bp updated
             if (y == i || y == bp) {
 #pragma unroll
                 for (int q = 0; q < CPT / 4; ++q) {
@@ -894,6 +907,7 @@ struct Round64Smem {
         } rb;
     } v;
     int ok;
+    int xj[2];                                       // local search: the entries of the current swap
     uint64_t tma_bar;                                // fused kernel: completion of the W tile copy
     __device__ __forceinline__ RoundView<64> view() {
         return RoundView<64>{a, u.gr.order, v.rb.rowbits, v.rb.bestv, v.rb.bestp, u.gr.rc, u.gr.cc, nullptr};
@@ -920,7 +934,7 @@ __device__ bool round_block_cta64(Key (&key)[32], Round64Smem<Key>& sm, int N, i
     __syncthreads();
     const bool ok = sm.ok;
     if (ok && sweeps > 0) {
-        local_search_mp<M>(sm.a, sm.u.bc, sm.u.bc + M * M, sh, sweeps, tid);
+        local_search_mp<M>(sm.a, sm.u.bc, sm.u.bc + M * M, sh, sm.xj, sweeps, tid);
         __syncthreads();
     }
     return ok;
