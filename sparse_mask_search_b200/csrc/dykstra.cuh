@@ -13,10 +13,11 @@
 //        C_j = sum_i e_ij N / R_i  c_j = log2 N - log2 C_j     (column step,
 //                                  reusing the row step's exponentials)
 //        y_ij += r_i + c_j                                     (clip folded in)
-//    so one exponential per entry and iteration, plus one log per row and
-//    one per column.
-//  * The plan is S = 2^min(y, 0) after the last iteration; S = 1 exactly
-//    for clipped entries (y >= 0).
+//    Written this way it takes one exponential per entry and iteration; the
+//    kernels below carry E = 2^y instead (row factors as clip thresholds,
+//    column factors on E) and take exponentials only at anchor points, see
+//    dykstra_tile_solve.
+//  * The plan is S = 2^min(y, 0) = min(E, 1) after the last iteration.
 //  * Since y only ever gains r_i + c_j, y = y0 + U_i + V_j with U, V the
 //    potentials accumulated so far: the 2M numbers (U, V) are the whole
 //    state of a block.  The EXT kernels start from given (U, V) (warm
