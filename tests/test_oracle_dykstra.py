@@ -10,7 +10,9 @@ and {S <= 1}.  The pins below do not restate the oracle's loop:
     the intersection (Bregman/Dykstra theory), characterised by its dual;
     the dual is minimised here by a generic quasi-Newton solver;
   - an independent linear-space (multiplicative) formulation of the same
-    iteration agrees at every finite iteration count;
+    iteration agrees at every finite iteration count, and so does the form
+    the kernels carry (row scalings as clip thresholds, column factors on
+    the exponentials, re-anchored from the accumulated potentials);
   - the entropic suboptimality bound 0 <= opt - <S,|W|> <= (m/tau) * F(S)
     with F(S) = -sum S log S <= N*M*log(M/N), which fixes the sign and the
     scale of tau in the kernel x0 = tau*|W|/max|W|.
@@ -112,6 +114,43 @@ def test_log_space_matches_linear_space(M, N, tau, iters):
     for a in oracle.blocks_view(np.abs(W), M).reshape(-1, M, M):
         S = oracle.block_plan(a, N, tau=tau, iters=iters)
         ref = linear_space_dykstra(a, N, tau, iters)
+        np.testing.assert_allclose(S, ref, rtol=0, atol=1e-9)
+
+
+def threshold_form_dykstra(a, N, tau, iters, anchor_every):
+    """The same iteration in the form the kernels carry it: the state is
+    y = y0 + U_i + V_j; between anchor points E = exp(y) = F / th_i, the row
+    step replaces the row's clip threshold th_i by S_i / N (S_i the row sum of
+    min(F, th_i)), the column step weighs min(F, th_i) by N / S_i and multiplies
+    F by N / C_j; at an anchor point the logarithms of the thresholds and of
+    the column factors' products move into U and V and F = exp(y0 + U + V)."""
+    M = a.shape[0]
+    y0 = kernel(a, tau) - tau
+    U = np.zeros(M); V = np.zeros(M)
+    F = np.exp(y0); th = np.ones(M); pv = np.ones(M)
+    for t in range(iters):
+        if t > 0 and t % anchor_every == 0:
+            U -= np.log(th); V += np.log(pv)
+            th = np.ones(M); pv = np.ones(M)
+            F = np.exp(y0 + U[:, None] + V[None, :])
+        e = np.minimum(F, th[:, None])
+        S_row = e.sum(axis=1)
+        C = (e * (N / S_row)[:, None]).sum(axis=0)
+        u = N / C
+        th = S_row / N
+        F = F * u[None, :]
+        pv = pv * u
+    return np.minimum(F / th[:, None], 1.0)
+
+
+@pytest.mark.parametrize("M,N,tau,iters", [(4, 2, 10.0, 200), (8, 4, 20.0, 200), (16, 8, 20.0, 300),
+                                           (32, 16, 20.0, 300), (64, 32, 30.0, 40)])
+@pytest.mark.parametrize("anchor_every", [1, 3, 64, 10 ** 9])
+def test_log_space_matches_threshold_form(M, N, tau, iters, anchor_every):
+    W = synth.random_blocks(3, M, seed=M + iters + 1, dist="t3_outlier_cols", dtype="bf16", scale=0.02)
+    for a in oracle.blocks_view(np.abs(W), M).reshape(-1, M, M):
+        S = oracle.block_plan(a, N, tau=tau, iters=iters)
+        ref = threshold_form_dykstra(a, N, tau, iters, anchor_every)
         np.testing.assert_allclose(S, ref, rtol=0, atol=1e-9)
 
 
