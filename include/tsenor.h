@@ -64,7 +64,8 @@ typedef enum {
     TSENOR_ERR_SHAPE = -2,           /* rows or cols negative or not a multiple of M */
     TSENOR_ERR_UNSUPPORTED_M = -3,   /* M not in {4, 8, 16, 32, 64} */
     TSENOR_ERR_CUDA = -4,            /* a CUDA runtime call failed; see tsenor_last_error() */
-    TSENOR_ERR_TOO_LARGE = -5        /* tsenor_mask_noalloc: rows*cols above TSENOR_NOALLOC_MAX_PARAMS */
+    TSENOR_ERR_DEVICE = -5,          /* tsenor_error_count: blocks failed on the device (count in *count_out) */
+    TSENOR_ERR_TOO_LARGE = -6        /* tsenor_mask_noalloc: rows*cols above TSENOR_NOALLOC_MAX_PARAMS */
 } tsenor_status;
 
 /*
@@ -113,7 +114,10 @@ tsenor_status tsenor_objective(const void* W, tsenor_dtype dtype, int64_t rows, 
 /*
  * Synchronises `stream`, then returns in *count_out the number of blocks that
  * failed on this device (non-finite input, or a rounding step that found no
- * move) since the previous call, and resets the counter.
+ * move) since the previous call, and resets the counter.  Returns TSENOR_OK
+ * when that number is 0 and TSENOR_ERR_DEVICE when it is not (the count is
+ * written in both cases); TSENOR_ERR_ARG for a null count_out, TSENOR_ERR_CUDA
+ * when the copy or the synchronisation fails.
  */
 tsenor_status tsenor_error_count(tsenor_stream_t stream, int64_t* count_out);
 
@@ -241,30 +245,37 @@ const char* tsenor_status_string(int status);
 const char* tsenor_last_error(void);
 
 /*
- * tsenor_mask_noalloc -- tsenor_mask for callers that must not allocate.
+ * tsenor_mask_noalloc -- the two-kernel plan + round path with its plan in
+ * a fixed array inside the library, for callers that cannot allocate.
  *
- * The TSENOR review has no counterpart of this entry point; it exists for
- * callers of this library that cannot let it allocate device memory:
+ * The TSENOR review has no counterpart of this entry point.  Running the
+ * plan and the rounding as two kernels (tsenor_plan, then tsenor_round) needs
+ * a rows x cols fp32 plan buffer between them, and some callers cannot
+ * allocate one at call time:
  *  - processes whose device memory is already reserved by another allocator
  *    (for example a framework's caching allocator holding most of the GPU),
- *    where a cudaMallocAsync inside the library can fail with out-of-memory
- *    although the caller still has free space in its own pool;
+ *    where a fresh cudaMalloc can fail with out-of-memory although the
+ *    caller still has free space in its own pool;
  *  - services that run under a fixed device-memory budget and must not grow
  *    their footprint, or wait on an allocation, while they are serving.
- *
- * Same arguments, results and error behaviour as tsenor_mask; the only
- * difference is where the plan between the two kernels lives.  Instead of a
- * stream-ordered cudaMallocAsync workspace, it uses a file-scope device array
- * of TSENOR_NOALLOC_MAX_PARAMS floats (64 MiB) inside the library.  That
- * array exists on every GPU that loads the library and stays allocated until
- * the process exits.  The call itself allocates nothing: no cudaMalloc,
+ * This entry point runs those two kernels with the plan in a file-scope
+ * device array of TSENOR_NOALLOC_MAX_PARAMS floats (64 MiB).  That array
+ * exists on every GPU that loads the library and stays allocated until the
+ * process exits.  The call itself allocates nothing: no cudaMalloc,
  * cudaMallocAsync, cudaFree or allocating library routine.
+ *
+ * Arguments, results and error behaviour are those of tsenor_mask, and the
+ * masks are equal bit for bit: tsenor_mask is one fused kernel that builds
+ * the same keys on chip (and allocates nothing either), so it is the faster
+ * call; this one takes the plan through device memory and back.
  *
  *  - rows * cols must not exceed TSENOR_NOALLOC_MAX_PARAMS; larger calls
  *    return TSENOR_ERR_TOO_LARGE before anything is enqueued.
  *  - The first call on a device looks up the array's device address on that
  *    device (cudaGetSymbolAddress, with the device current) and keeps it for
- *    later calls; make that first call before any stream capture.
+ *    later calls; it is looked up again when the device's current context
+ *    has changed (after a cudaDeviceReset, for example).  Make the first call
+ *    on each device before any stream capture.
  *  - Every call on a device shares the one array, and the array keeps the
  *    last call's contents.  Nothing in it needs to start at zero: each call
  *    writes the whole plan region it later reads.  Calls whose work overlaps

@@ -22,8 +22,7 @@
  * while its row and column budgets remain, then swap entries in with the
  * 2-in/1-out move scored (|W_ij'| + |W_i'j|) - |W_i'j'|.
  *
- * Readings taken where the pages leave a step open (each is also listed in
- * the design notes):
+ * Readings taken where the pages leave a step open:
  *  - kernel: x0_ij = tau * a_ij / max(a over the block), x0 = 0 for an
  *    all-zero block; logQ0 = 0.
  *  - one iteration = row step, column step, clip; only the clip carries a
@@ -35,8 +34,19 @@
  *  - repair: while a row is short, take the lowest short row i and the lowest
  *    short column j and apply the 2-in/1-out move with the best score,
  *    whatever its sign (ties: lowest i'*M + j').  With the full greedy scan a
- *    candidate always exists (proof in the design notes); if none did, the
- *    block is reported as failed.
+ *    candidate always exists; the block is reported as failed only if none
+ *    does (never expected).  Why one exists: the greedy visits every entry,
+ *    so when it ends every pair (short row i, short column j) is taken --
+ *    entry (i,j) was visited while both still had budget.  A short row
+ *    exists only if a short column does (rows and columns hold the same
+ *    number of ones), and column j short means some row i' has s_i'j = 0;
+ *    such a row is full (N ones), for otherwise (i',j) would be a short
+ *    pair that is not taken.  Row i is short, so it has at least M-N+1
+ *    zeros, and N + (M-N+1) > M: some column j' holds a one of row i' and a
+ *    zero of row i, and (i,j'),(i',j) in, (i',j') out is a candidate.  A
+ *    move takes a one only from a full row and adds ones to row i and
+ *    column j, so "every short row x short column pair is taken" still holds
+ *    after it, and the argument repeats until no row is short.
  *  - local search: one sweep visits anchor rows i = 0..M-1; for each anchor
  *    the best partner row i' is chosen by the net gain of freeing (i,j) and
  *    taking the 2-in/1-out move, and the move is applied only if that gain is

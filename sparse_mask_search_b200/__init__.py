@@ -14,7 +14,7 @@ LIB_PATH = os.path.join(HERE, "libtsenor_b200.so")
 
 TSENOR_F32, TSENOR_BF16 = 0, 1
 STATUS = {0: "TSENOR_OK", -1: "TSENOR_ERR_ARG", -2: "TSENOR_ERR_SHAPE", -3: "TSENOR_ERR_UNSUPPORTED_M",
-          -4: "TSENOR_ERR_CUDA", -5: "TSENOR_ERR_TOO_LARGE"}
+          -4: "TSENOR_ERR_CUDA", -5: "TSENOR_ERR_DEVICE", -6: "TSENOR_ERR_TOO_LARGE"}
 NOALLOC_MAX_PARAMS = 16 * 1024 * 1024
 EXPORTS = ("tsenor_mask", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
            "tsenor_status_string", "tsenor_last_error", "tsenor_mask_noalloc", "tsenor_mask_safeguard",
@@ -289,9 +289,15 @@ def tsenor_objective(W, mask, N: int, M: int, out=None, stream=None):
 
 
 def tsenor_error_count(stream=None) -> int:
-    """Blocks that failed since the previous call (synchronises the stream)."""
+    """Blocks that failed since the previous call (synchronises the stream).
+
+    The C call reports a nonzero count with TSENOR_ERR_DEVICE; here the count
+    itself is the result, so that status is not raised.
+    """
     n = C.c_int64(0)
-    _check(lib().tsenor_error_count(_stream_handle(stream), C.byref(n)))
+    status = lib().tsenor_error_count(_stream_handle(stream), C.byref(n))
+    if status != -5:
+        _check(status)
     return int(n.value)
 
 

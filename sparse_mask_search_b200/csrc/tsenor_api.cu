@@ -528,7 +528,7 @@ extern "C" tsenor_status tsenor_error_count(tsenor_stream_t stream, int64_t* cou
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e, "tsenor_error_count");
     *count_out = int64_t(v);
-    return TSENOR_OK;
+    return v ? TSENOR_ERR_DEVICE : TSENOR_OK;
 }
 
 extern "C" const char* tsenor_status_string(int status) {
@@ -538,6 +538,7 @@ extern "C" const char* tsenor_status_string(int status) {
         case TSENOR_ERR_SHAPE: return "rows/cols not a non-negative multiple of M";
         case TSENOR_ERR_UNSUPPORTED_M: return "M must be 4, 8, 16, 32 or 64";
         case TSENOR_ERR_CUDA: return "CUDA runtime error";
+        case TSENOR_ERR_DEVICE: return "blocks failed on the device (non-finite input or no repair move); see the count";
         case TSENOR_ERR_TOO_LARGE: return "rows*cols exceeds TSENOR_NOALLOC_MAX_PARAMS (16777216) of tsenor_mask_noalloc";
         default: return "unknown status";
     }
@@ -546,11 +547,14 @@ extern "C" const char* tsenor_status_string(int status) {
 extern "C" const char* tsenor_last_error(void) { return tsenor::g_last_error; }
 
 // ---------------------------------------------------------------------------
-// tsenor_mask_noalloc: the plan between the two kernels lives in a file-scope
-// device array instead of a cudaMallocAsync workspace (see include/tsenor.h).
-// Host code must not hand `g_noalloc_plan` itself to a kernel: on the host
-// that name is only a stand-in for the symbol, not a device address.  The
-// device address is looked up once per device with cudaGetSymbolAddress.
+// tsenor_mask_noalloc: the plan + round kernels with the plan between them
+// in a file-scope device array, so that the call allocates nothing (see
+// include/tsenor.h).  Host code must not hand `g_noalloc_plan` itself to a
+// kernel: on the host that name is only a stand-in for the symbol, not a
+// device address.  The device address is looked up with
+// cudaGetSymbolAddress once per device and context: the cache is keyed by
+// the context that is current on the device, so a new primary context
+// (after cudaDeviceReset) gets a fresh lookup.
 
 static __device__ __align__(256) float g_noalloc_plan[TSENOR_NOALLOC_MAX_PARAMS];
 
@@ -558,19 +562,36 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 float* g_noalloc_ptr[kMaxDevices] = {};
+CUcontext g_noalloc_ctx[kMaxDevices] = {};
+PFN_cuCtxGetCurrent g_ctx_current = nullptr;
+std::once_flag g_ctx_once;
 
-// Device address of g_noalloc_plan on the current device (first call per device looks it up).
+// Device address of g_noalloc_plan on the current device and context.
 cudaError_t noalloc_plan_ptr(float** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::call_once(g_ctx_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent>(fn);
+    });
+    if (!g_ctx_current) return cudaErrorNotSupported;
+    // no current context yet on this thread (the runtime makes the primary
+    // context current lazily): the symbol lookup below does that first
+    CUcontext ctx = nullptr;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+    if (!g_noalloc_ptr[dev] || !ctx || g_noalloc_ctx[dev] != ctx) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_plan);
         if (e != cudaSuccess) return e;
+        if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
         g_noalloc_ptr[dev] = static_cast<float*>(p);
+        g_noalloc_ctx[dev] = ctx;
     }
     *out = g_noalloc_ptr[dev];
     return cudaSuccess;

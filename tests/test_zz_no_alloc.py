@@ -1,9 +1,9 @@
-"""tsenor_mask_noalloc: the entry point for callers that cannot let the library
-allocate device memory (their memory is held by another allocator, or they run
-under a fixed device-memory budget).  It keeps the plan in an array inside the
-library instead of a cudaMallocAsync workspace, so its masks must equal
-tsenor_mask's bit for bit (masks are integer results), call after call, even
-though every call reuses the same array.
+"""tsenor_mask_noalloc: the plan + round kernels with the plan between them
+in a fixed array inside the library, for callers that cannot allocate device
+memory at call time (their memory is held by another allocator, or they run
+under a fixed device-memory budget).  Its masks must equal tsenor_mask's bit
+for bit (masks are integer results), call after call, even though every call
+reuses the same array.
 
 Collected last on purpose: if it fails, a run that stops at the first failure
 has already run every other test.
@@ -60,6 +60,6 @@ def test_noalloc_rejects_sizes_above_its_array():
     rows, cols = 8192, 4096          # 2 * 16 Mi params: rejected on the host before any launch
     status = L.tsenor_mask_noalloc(C.c_void_p(Wd.data_ptr()), tsl.TSENOR_BF16, rows, cols, 2, 4, 10.0, 5, 1,
                                    C.c_void_p(out.data_ptr()), None)
-    assert status == -5
+    assert status == -6
     assert b"TSENOR_NOALLOC_MAX_PARAMS" in L.tsenor_status_string(status)
     assert rows * cols > tsl.NOALLOC_MAX_PARAMS
