@@ -27,7 +27,7 @@
  *    passed in its place.  rows and cols must be multiples of M (the review leaves other
  *    shapes open, "Assumptions & free parameters"); rows == 0 or cols == 0
  *    is a valid empty call that does nothing.
- *  - Supported M: 4, 8, 16, 32, 64.  1 <= N <= M.  tau > 0 and finite,
+ *  - Supported M: 4, 8, 16, 32, 64.  1 <= N <= M.  0 < tau <= TSENOR_MAX_TAU,
  *    iters >= 1, sweeps >= 0.
  *  - The kernel of block b is x0_ij = tau * |W_ij| / max(|W| over b)
  *    (x0 = 0 for an all-zero block); one iteration is a row step, a column
@@ -58,9 +58,20 @@ typedef struct CUstream_st* tsenor_stream_t;   /* same type as cudaStream_t */
 
 typedef enum { TSENOR_F32 = 0, TSENOR_BF16 = 1 } tsenor_dtype;
 
+/*
+ * Largest tau accepted (larger values return TSENOR_ERR_ARG).  The kernels
+ * carry the exponentials of the Dykstra state in fp32, and a block's kernel
+ * exp(tau * |W| / max|W|) spans a factor 2^(tau * log2 e) between its
+ * smallest and largest entry; at tau = 80 that is 2^115, inside the normal
+ * fp32 range with room for the potentials.  The review's default
+ * temperature, 0.005 * max|W| ("Assumptions & free parameters"), corresponds
+ * to tau = 200 in this convention and is outside it.
+ */
+#define TSENOR_MAX_TAU 80.0f
+
 typedef enum {
     TSENOR_OK = 0,
-    TSENOR_ERR_ARG = -1,             /* null pointer, bad dtype, N/tau/iters/sweeps out of range, misaligned pointer */
+    TSENOR_ERR_ARG = -1,             /* null pointer, bad dtype, N/tau/iters/sweeps out of range (tau: see TSENOR_MAX_TAU), misaligned pointer */
     TSENOR_ERR_SHAPE = -2,           /* rows or cols negative or not a multiple of M */
     TSENOR_ERR_UNSUPPORTED_M = -3,   /* M not in {4, 8, 16, 32, 64} */
     TSENOR_ERR_CUDA = -4,            /* a CUDA runtime call failed; see tsenor_last_error() */

@@ -16,6 +16,7 @@ TSENOR_F32, TSENOR_BF16 = 0, 1
 STATUS = {0: "TSENOR_OK", -1: "TSENOR_ERR_ARG", -2: "TSENOR_ERR_SHAPE", -3: "TSENOR_ERR_UNSUPPORTED_M",
           -4: "TSENOR_ERR_CUDA", -5: "TSENOR_ERR_DEVICE", -6: "TSENOR_ERR_TOO_LARGE"}
 NOALLOC_MAX_PARAMS = 16 * 1024 * 1024
+MAX_TAU = 80.0            # TSENOR_MAX_TAU: larger tau is rejected (TSENOR_ERR_ARG)
 EXPORTS = ("tsenor_mask", "tsenor_plan", "tsenor_round", "tsenor_objective", "tsenor_error_count",
            "tsenor_status_string", "tsenor_last_error", "tsenor_mask_noalloc", "tsenor_mask_safeguard",
            "tsenor_mask_padded", "tsenor_mask_warm", "tsenor_plan_warm", "tsenor_mask_scores", "tsenor_mask_host")

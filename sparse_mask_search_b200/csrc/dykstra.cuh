@@ -15,8 +15,8 @@
 //        y_ij += r_i + c_j                                     (clip folded in)
 //    Written this way it takes one exponential per entry and iteration; the
 //    kernels below carry E = 2^y instead (row factors as clip thresholds,
-//    column factors on E) and take exponentials only at anchor points, see
-//    dykstra_tile_solve.
+//    column factors on E) and rebuild it only at anchor points, as
+//    E = 2^y0 * 2^U_i * 2^V_j, see dykstra_tile_solve.
 //  * The plan is S = 2^min(y, 0) = min(E, 1) after the last iteration.
 //  * Since y only ever gains r_i + c_j, y = y0 + U_i + V_j with U, V the
 //    potentials accumulated so far: the 2M numbers (U, V) are the whole
@@ -30,6 +30,7 @@
 
 #include <type_traits>
 
+#include "../../include/tsenor.h"
 #include "common.cuh"
 #include "tma.cuh"
 
@@ -51,6 +52,34 @@ struct DykstraExt {
 // (see dykstra_tile_solve).
 constexpr int kAnchorEvery = 64;
 
+// Largest tau the kernels accept (TSENOR_MAX_TAU; the host rejects larger
+// ones): E0 = 2^y0 spans 2^-tau2 .. 1 within a block (tau2 = tau * log2(e)),
+// which must stay inside the normal fp32 range; at tau = 80, tau2 = 115.4.
+constexpr float kMaxTau = TSENOR_MAX_TAU;
+
+// 2^y for a double y in [-126, 126] (clamped), as fp32, to within the
+// hardware exponential's error: y = n + f with n the nearest integer (the
+// 1.5 * 2^52 shift leaves n in the low word of the sum) and |f| <= 1/2, so
+// the fp32 rounding of f costs at most 2^-26 in the exponent, and 2^n is an
+// exact scaling.  Used where the exponent is large but its result must be
+// good to a few ulps: E0 = 2^y0 and the potentials' factors 2^U, 2^V.
+__device__ __forceinline__ float exp2_wide(double y) {
+    y = fmin(fmax(y, -126.0), 126.0);
+    constexpr double kShift = 6755399441055744.0;    // 1.5 * 2^52
+    const double s = y + kShift;
+    const int n = __double2loint(s);
+    const float f = __double2float_rn(y - (s - kShift));
+    return ex2(f) * __int_as_float((n + 127) << 23);
+}
+
+
+// E0 = 2^y0 of one entry, y0 = tau2 (a / max|W| - 1) in fp64.  Out of line:
+// inlined 64 times into the one-thread-per-block solver (M = 8) it made the
+// compiler keep many fp64 temporaries live at once and spill the solver's
+// registers; as a call it costs a few instructions per entry, once.
+__device__ __noinline__ float e0_of(double tau2d, float a, double inv_m) {
+    return exp2_wide(fma(tau2d, double(a) * inv_m, -tau2d));
+}
 
 // ---------------------------------------------------------------------------
 // M = 4, 8: one thread holds a whole block in registers.  Rows are streamed:
@@ -70,11 +99,11 @@ __device__ __forceinline__ float4 lds4_keep(const float* p) {
 // dykstra_tile_solve: the state is y = y0 + U_i + V_j, E = 2^y = F / TH_i is
 // carried in linear form between anchor points (the row step sets the row's
 // clip threshold TH_i, the column step multiplies F by N / C_j) and
-// recomputed from y0 + U + V every kAnchorEvery iterations, when the
-// logarithms of the thresholds and of the column factors' products are added
-// to U and V (fp32), so the potentials follow the very factors applied.
-// y0s: this thread's M*M floats of shared memory (16-byte aligned), which
-// hold y0 during the iterations.  On return `s` holds the plan
+// recomputed every kAnchorEvery iterations as (E0_ij * 2^U_i) * 2^V_j with
+// E0 = 2^y0, when the logarithms of the thresholds and of the column factors'
+// products are added to U and V (fp32), so the potentials follow the very
+// factors applied.  y0s: this thread's M*M floats of shared memory (16-byte
+// aligned), which hold E0 during the iterations.  On return `s` holds the plan
 // 2^min(y, 0); returns whether the block's W is finite.
 template <int M, typename T, bool EXT = false>
 __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* __restrict__ W, int64_t cols,
@@ -102,14 +131,13 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
             finite = finite && (y[i][j] <= 3.402823466e38f);   // false for NaN and Inf
             m = fmaxf(m, y[i][j]);
         }
-    const float tau2 = tau * kLog2e;
+    // y0 in fp64 (as the oracle's x0), kept as E0 = 2^y0
+    const double tau2d = double(tau) * kLog2eD;
+    const double inv_m = m > 0.f ? 1.0 / double(m) : 0.0;
 #pragma unroll
     for (int i = 0; i < M; ++i) {
 #pragma unroll
-        for (int j = 0; j < M; ++j) {
-            const float q = m > 0.f ? __fdiv_rn(y[i][j], m) : 0.f;
-            y[i][j] = fmaf(tau2, q, -tau2);
-        }
+        for (int j = 0; j < M; ++j) y[i][j] = e0_of(tau2d, y[i][j], inv_m);
 #pragma unroll
         for (int v = 0; v < M / 4; ++v)
             reinterpret_cast<float4*>(y0s + i * M)[v] = make_float4(y[i][4 * v], y[i][4 * v + 1], y[i][4 * v + 2],
@@ -146,27 +174,55 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
     // column pairs (j, j+1) as packed fp32x2 values
     constexpr int M2 = M / 2;
     float2 E2[M][M2];                                // F
+    // F = 2^(y0 + U_i + V_j) = (E0_ij * 2^U_i) * 2^V_j, so that the rounding
+    // of the large potentials is common to a row or a column.  The factors
+    // stay in the fp32 range while every |U_i|, |V_j| is below 124 (from a
+    // cold start they stay within about tau * log2(e) + log2(M) <= 122); a
+    // warm start from potentials beyond that takes the exponent
+    // lg2(E0) + U_i + V_j per entry instead.
     auto anchor = [&]() {
         flush();
+        float span = 0.f;
 #pragma unroll
-        for (int k = 0; k < M; ++k) TH[k] = 1.f;
+        for (int k = 0; k < M; ++k) {
+            TH[k] = 1.f;
+            span = fmaxf(span, fmaxf(fabsf(U[k]), fabsf(V[k])));
+        }
+        if (span < 124.f) {
+            float2 Q2v[M2];
 #pragma unroll
-        for (int i = 0; i < M; ++i)
+            for (int c = 0; c < M2; ++c) Q2v[c] = make_float2(ex2(V[2 * c]), ex2(V[2 * c + 1]));
 #pragma unroll
-            for (int v = 0; v < M / 4; ++v) {
-                const float4 q = lds4_keep(y0s + i * M + 4 * v);
-                const float2 u2 = make_float2(U[i], U[i]);
-                const float2 a = add2(make_float2(q.x, q.y), add2(u2, make_float2(V[4 * v], V[4 * v + 1])));
-                const float2 c = add2(make_float2(q.z, q.w), add2(u2, make_float2(V[4 * v + 2], V[4 * v + 3])));
-                E2[i][2 * v] = make_float2(ex2(a.x), ex2(a.y));
-                E2[i][2 * v + 1] = make_float2(ex2(c.x), ex2(c.y));
+            for (int i = 0; i < M; ++i) {
+                const float p = ex2(U[i]);
+                const float2 p2 = make_float2(p, p);
+#pragma unroll
+                for (int v = 0; v < M / 4; ++v) {
+                    const float4 q = lds4_keep(y0s + i * M + 4 * v);
+                    E2[i][2 * v] = mul2(mul2(make_float2(q.x, q.y), p2), Q2v[2 * v]);
+                    E2[i][2 * v + 1] = mul2(mul2(make_float2(q.z, q.w), p2), Q2v[2 * v + 1]);
+                }
             }
+        } else {
+#pragma unroll
+            for (int i = 0; i < M; ++i)
+#pragma unroll
+                for (int v = 0; v < M / 4; ++v) {
+                    const float4 q = lds4_keep(y0s + i * M + 4 * v);
+                    E2[i][2 * v] = make_float2(ex2(lg2(q.x) + (U[i] + V[4 * v])), ex2(lg2(q.y) + (U[i] + V[4 * v + 1])));
+                    E2[i][2 * v + 1] = make_float2(ex2(lg2(q.z) + (U[i] + V[4 * v + 2])),
+                                                   ex2(lg2(q.w) + (U[i] + V[4 * v + 3])));
+                }
+        }
     };
-    anchor();
+    // one call site, at the top of each anchor period: with a second call
+    // before the loop the compiler laid the loop out slower (A/B: one 4:8
+    // matrix 0.93 -> 1.00 ms, the 16:32 plan kernel 2.11 -> 2.64 ms); the
+    // result is unused for a non-finite block, which runs no period
     bool stop = !finite;
 #pragma unroll 1
     for (int t0 = 0; t0 < iters && !stop; t0 += kAnchorEvery) {
-        if (t0 > 0) anchor();
+        anchor();
         const int t1 = min(iters, t0 + kAnchorEvery);
 #pragma unroll 1
         for (int t = t0; t < t1; ++t) {
@@ -357,7 +413,12 @@ struct TileSource {
 // iterations log2 of the threshold and of the column factors' product are
 // added to U and V, and E is re-anchored to 2^(y0 + U + V) (th = 1), so that
 // an entry that underflowed for a while recovers and the rounding of the
-// products never builds up.
+// products never builds up.  The anchor is taken as the product
+// (E0_ij * 2^U_i) * 2^V_j, E0 = 2^y0 computed once from an fp64 y0: y0 and
+// U + V are each of size up to tau * log2(e) and cancel, so their fp32 sum
+// would put an error of about |y0| * 2^-24 into every entry, which the
+// iterations do not remove; in the product form each entry carries a few
+// ulps, and the rounding of a potential is common to its row or column.
 
 // EXT: warm start from / export to ext.potentials of block b, stop rule
 // ext.tol2, iteration count to ext.iters_used.
@@ -465,20 +526,22 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
         m = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
         finite = red_f[0] && red_f[1] && red_f[2] && red_f[3];
     }
-    // y0 = (x0 - tau) log2 e with x0 = tau |W| / max|W|, kept in the tile
-    // for the anchor points: column pair (k, c) of thread t at float2 slot
+    // y0 = (x0 - tau) log2 e with x0 = tau |W| / max|W|, taken in fp64 (as
+    // the oracle's x0); kept in the tile for the anchor points as E0 = 2^y0:
+    // column pair (k, c) of thread t at float2 slot
     // (k * Q/2 + c) * TPB + t (consecutive threads, consecutive slots)
     block_sync();                                    // every thread has read its |W|
-    const float tau2 = tau * kLog2e;
+    const double tau2d = double(tau) * kLog2eD;
+    const double inv_m = m > 0.f ? 1.0 / double(m) : 0.0;
     float2* y0t = reinterpret_cast<float2*>(tile) + th.t;
     static_assert(P * Q * C::TPB <= M * TS, "y0 fits the tile");
 #pragma unroll
     for (int k = 0; k < P; ++k)
 #pragma unroll
         for (int c = 0; c < Q2; ++c) {
-            const float q0 = m > 0.f ? __fdiv_rn(y[k][2 * c], m) : 0.f;
-            const float q1 = m > 0.f ? __fdiv_rn(y[k][2 * c + 1], m) : 0.f;
-            y0t[(k * Q2 + c) * C::TPB] = make_float2(fmaf(tau2, q0, -tau2), fmaf(tau2, q1, -tau2));
+            const double y0a = fma(tau2d, double(y[k][2 * c]) * inv_m, -tau2d);
+            const double y0b = fma(tau2d, double(y[k][2 * c + 1]) * inv_m, -tau2d);
+            y0t[(k * Q2 + c) * C::TPB] = make_float2(exp2_wide(y0a), exp2_wide(y0b));
         }
     const float fN = float(N);
 
@@ -511,17 +574,20 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
 #pragma unroll
         for (int lo = 0; lo < C::CO; ++lo) va[lo] = uv ? double(uv[M + th.col(lo)]) * kLog2eD : 0.0;
     }
-    // F = E = 2^(y0 + U_i + V_j) over this thread's entries and th = 1 (the
-    // potentials, rounded to fp32, all-gathered from their owners into the
-    // permuted register order)
+    // F = E = 2^(y0 + U_i + V_j) = (E0_ij * 2^U_i) * 2^V_j over this thread's
+    // entries and th = 1, the factors taken from the fp64 potentials by their
+    // owners and all-gathered into the permuted register order; the
+    // potentials' large magnitudes (up to about tau2) never meet in an fp32
+    // sum, so each entry carries only a few ulps of rounding, and an error in
+    // a factor is common to a whole row or column.
     float2 F2[P][Q2];                                // column pairs packed
     auto anchor = [&]() {
         flush();
 #pragma unroll
         for (int k = 0; k < P; ++k) thr[k] = 1.f;
-        float U[P], V[Q];
+        float U[P], V[Q];                            // 2^U_i, 2^V_j
 #pragma unroll
-        for (int lo = 0; lo < C::RO; ++lo) U[lo] = float(ua[lo]);
+        for (int lo = 0; lo < C::RO; ++lo) U[lo] = exp2_wide(ua[lo]);
 #pragma unroll
         for (int s = 1; s < C::RSR; s <<= 1)
 #pragma unroll
@@ -530,7 +596,7 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
                 for (int lo = 0; lo < C::RO; ++lo)
                     U[(hi + s) * C::RO + lo] = __shfl_xor_sync(kFullMask, U[hi * C::RO + lo], s);
 #pragma unroll
-        for (int lo = 0; lo < C::CO; ++lo) V[lo] = float(va[lo]);
+        for (int lo = 0; lo < C::CO; ++lo) V[lo] = exp2_wide(va[lo]);
 #pragma unroll
         for (int s = 1; s < C::RSC; s <<= 1)
 #pragma unroll
@@ -541,13 +607,10 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
 #pragma unroll
         for (int k = 0; k < P; ++k)
 #pragma unroll
-            for (int c = 0; c < Q2; ++c) {
-                const float2 uv2 = add2(make_float2(U[k], U[k]), make_float2(V[2 * c], V[2 * c + 1]));
-                const float2 y2 = add2(lds_keep(y0t + (k * Q2 + c) * C::TPB), uv2);
-                F2[k][c] = make_float2(ex2(y2.x), ex2(y2.y));
-            }
+            for (int c = 0; c < Q2; ++c)
+                F2[k][c] = mul2(mul2(lds_keep(y0t + (k * Q2 + c) * C::TPB), make_float2(U[k], U[k])),
+                                make_float2(V[2 * c], V[2 * c + 1]));
     };
-    anchor();
     bool done = !finite;                             // EXT: this block has stopped
     int used = 0;
 
@@ -558,7 +621,7 @@ __device__ __forceinline__ bool dykstra_tile_solve(const TileSource<T>& src, int
     bool stop = !run;
 #pragma unroll 1
     for (int it0 = 0; it0 < iters && !stop; it0 += kAnchorEvery) {
-        if (it0 > 0) anchor();
+        anchor();                                    // one call site (see dykstra_thread_solve)
         const int it1 = min(iters, it0 + kAnchorEvery);
 #pragma unroll 1
         for (int it = it0; it < it1; ++it) {

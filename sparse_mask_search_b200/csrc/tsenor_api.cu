@@ -248,7 +248,7 @@ cudaError_t run_round(int dtype, int M, const float* plan, const void* W, int64_
 }
 
 bool solver_params_ok(float tau, int iters) {
-    return tau > 0.f && tau <= 3.0e38f && iters >= 1;
+    return tau > 0.f && tau <= kMaxTau && iters >= 1;
 }
 
 // Arguments of the warm-start entry points beyond the plain ones.

@@ -7,7 +7,10 @@ import numpy as np
 import oracle
 
 PLAN_TOL = 1e-4          # max |S_gpu - S_oracle| (fp32 plan vs fp64 plan)
-NEAR_TIE = 2e-4          # a block may differ only through pairs whose oracle keys lie this close
+# A block may differ from the oracle's only through a near-tie: every pair of
+# entries that the two key sets order differently has oracle keys within this
+# relative distance, |S_e - S_f| / max(S_e, S_f).
+NEAR_TIE = 1e-6
 
 
 def to_device(storage, dtype):
@@ -32,7 +35,8 @@ def order(S, a):
 
 
 def max_inverted_gap(S_ref, S_gpu, a):
-    """Largest |S_ref[e] - S_ref[f]| over entry pairs that the two key sets order differently."""
+    """Largest relative gap |S_ref[e] - S_ref[f]| / max(S_ref[e], S_ref[f]) over the
+    entry pairs that the two key sets order differently (0 when none is)."""
     o = order(S_ref, a)
     pos = np.empty(S_ref.size, dtype=np.int64)
     pos[order(S_gpu, a)] = np.arange(S_ref.size)
@@ -44,8 +48,10 @@ def max_inverted_gap(S_ref, S_gpu, a):
         u = np.arange(u0, min(E, u0 + 512))
         inv = (P[u][:, None] > P[None, :]) & (u[:, None] < np.arange(E)[None, :])
         if inv.any():
-            d = np.abs(ks[u][:, None] - ks[None, :])[inv]
-            best = max(best, float(d.max()))
+            d = np.abs(ks[u][:, None] - ks[None, :])
+            scale = np.maximum(np.abs(ks[u][:, None]), np.abs(ks[None, :]))
+            rel = np.divide(d, scale, out=np.zeros_like(d), where=scale > 0)
+            best = max(best, float(rel[inv].max()))
     return best
 
 

@@ -32,9 +32,19 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings():
     L = tsl.lib()
-    for code in (0, -1, -2, -3, -4):
-        assert L.tsenor_status_string(code)
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert L.tsenor_status_string(code) != b"unknown status"
     assert L.tsenor_last_error() == b""
+
+
+def test_largest_tau_is_accepted_up_to_the_documented_limit():
+    # the header's TSENOR_MAX_TAU and the binding's copy agree; tau = 80 passes the
+    # checks (the empty call returns before any launch), 80.5 does not
+    text = open(os.path.join(ROOT, "include", "tsenor.h")).read()
+    assert float(re.search(r"#define TSENOR_MAX_TAU ([0-9.]+)f", text).group(1)) == tsl.MAX_TAU == 80.0
+    L = tsl.lib()
+    assert _mask(L, rows=0, W=0, out=0, tau=80.0) == 0
+    assert _mask(L, rows=0, W=0, out=0, tau=80.5) == -1
 
 
 def _mask(L, W=1 << 12, dtype=1, rows=64, cols=64, N=2, M=4, tau=10.0, iters=5, sweeps=1, out=1 << 12):
@@ -46,6 +56,7 @@ def _mask(L, W=1 << 12, dtype=1, rows=64, cols=64, N=2, M=4, tau=10.0, iters=5, 
     (dict(N=0), -1), (dict(N=5), -1),
     (dict(rows=66), -2), (dict(cols=-4), -2),
     (dict(tau=0.0), -1), (dict(tau=float("nan")), -1), (dict(tau=float("inf")), -1),
+    (dict(tau=80.5), -1), (dict(tau=200.0), -1),
     (dict(iters=0), -1), (dict(sweeps=-1), -1),
     (dict(dtype=7), -1),
     (dict(W=0), -1), (dict(W=(1 << 12) + 2), -1),

@@ -13,6 +13,40 @@ def test_fp32_peak_from_unit_counts_and_clock():
     assert bench.fp32_peak_tops(1965.0) == pytest.approx(37.22, abs=0.01)
 
 
+def test_roofline_fractions_follow_the_survey_count_and_the_fma_count():
+    # the 4096 x 11008 16:32 workload (T = 300) at 3.529 ms per call, against
+    # the unit-count peaks at 1965 MHz: MUFU 148 x 16, FP32 148 x 128 per clock
+    params, M, T, ms = 4096 * 11008, 32, 300, 3.529
+    peaks = {"fma_tops": bench.fp32_peak_tops(1965.0), "mufu_tops": bench.mufu_peak_tops(1965.0)}
+    assert peaks["mufu_tops"] == pytest.approx(148 * 16 * 1965e6 / 1e12)
+    r = bench.roofline_record(params, M, T, ms, peaks)
+    t = ms / 1e3
+    mufu = params * T * (1 + 2 / M) / (peaks["mufu_tops"] * 1e12) / t     # 318.75 ex2/lg2 per param
+    fp32 = params * T * 8 / (peaks["fma_tops"] * 1e12) / t
+    fma = params * T * 3 / (peaks["fma_tops"] * 1e12) / t
+    assert r["frac_survey"]["mufu"] == pytest.approx(mufu) and mufu == pytest.approx(0.875, abs=0.001)
+    assert r["frac_survey"]["fp32"] == pytest.approx(fp32) and fp32 == pytest.approx(0.824, abs=0.001)
+    assert r["frac_fma"] == pytest.approx(fma) and fma == pytest.approx(0.309, abs=0.001)
+    # the slower roofline binds: the MUFU one here, and `frac` is its fraction
+    assert r["binding_pipe"] == "mufu"
+    assert r["frac"] == pytest.approx(r["frac_survey"]["binding"]) and r["frac"] == pytest.approx(mufu)
+    assert r["achieved"] / r["peak"] == pytest.approx(r["frac"])
+    # with a slow FP32 pipe the FP32 roofline binds instead
+    r2 = bench.roofline_record(params, M, T, ms, {"fma_tops": 10.0, "mufu_tops": peaks["mufu_tops"]})
+    assert r2["binding_pipe"] == "fp32" and r2["frac"] == pytest.approx(r2["frac_survey"]["fp32"])
+
+
+def test_clock_window_summary():
+    cs = object.__new__(bench.ClockSampler)
+    cs.max_mhz = 1965.0
+    cs.samples = [(0.000, 1965.0, 0x0, 300.0), (0.002, 1950.0, 0x4, None), (0.004, 1965.0, 0x0, None),
+                  (0.050, 900.0, 0x40, 500.0)]
+    w = cs.window(0.0, 0.005)
+    assert w["samples"] == 3 and w["sm_mhz"] == 1965.0 and w["sm_mhz_min"] == 1950.0
+    assert w["reasons"] == ["sw_power_cap"] and w["power_w_max"] == 300.0
+    assert cs.window(0.0, 0.06)["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+
+
 def test_workload_shape_override():
     args = bench.parse_args(["--workload", "w8192x28672_bf16_laplace_32of64", "--shape", "2048x8192"])
     w = bench.workload_of(args)

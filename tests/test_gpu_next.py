@@ -152,6 +152,6 @@ def test_offsets_beyond_int32(M, N):
             A = oracle.blocks_view(np.abs(sub), M)
             for c in np.nonzero(~same)[0]:
                 assert max_inverted_gap(Pr[0, c], Pg[0, c], A[0, c]) <= NEAR_TIE, (r0, c)
-        assert same.mean() >= 0.99
+        assert same.mean() >= 0.999
     del Wd, mask, obj
     torch.cuda.empty_cache()

@@ -130,6 +130,23 @@ def test_full_256x256_2of4():
     check_pipeline(w.name, stor, W, w.dtype, w.N, w.M, w.tau, w.iters, w.sweeps)
 
 
+@pytest.mark.parametrize("M,N,dtype", [(8, 4, "f32"), (16, 8, "bf16"), (32, 16, "bf16"), (64, 32, "bf16")])
+def test_largest_tau(M, N, dtype):
+    """tau = 80 (the largest accepted): the block's kernel spans 2^115, near the edge
+    of the fp32 range the linear-form exponentials live in.  Plan within the plan
+    bar; masks valid and equal to the oracle's but for near-ties."""
+    rows, cols = 2 * M, 8 * M
+    stor, W = synth.make_matrix(rows, cols, dtype, "laplace_outliers", 0.02, seed=500 + M)
+    check = (M, N, dtype, rows, cols, 80.0, 300, 4, "laplace_outliers")
+    Wd = to_device(stor, dtype)
+    P_gpu = tsl.tsenor_plan(Wd, N, M, 80.0, 300).cpu().numpy()
+    P_ref = oracle.plan(W, N, M, 80.0, 300)
+    assert np.abs(P_gpu.astype(np.float64) - P_ref).max() <= PLAN_TOL
+    check_pipeline("mask_tau80_" + _ids(check), stor, W, dtype, N, M, 80.0, 300, 4, min_identical=0.0)
+    with pytest.raises(tsl.TsenorError):
+        tsl.tsenor_mask(Wd, N, M, 80.5, 300, 4)
+
+
 def test_objective_matches_oracle_on_oracle_masks():
     stor, W = synth.make_matrix(64, 128, "bf16", "normal", 0.02, seed=3)
     m_ref, _, _ = oracle.mask(W, 8, 16, 20.0, 50, 2)

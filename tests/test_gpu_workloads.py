@@ -1,10 +1,12 @@
 """Full-size workloads, in the launch configuration the benchmark times.
 
 Every block of the full matrix is checked for validity on the device
-(tsenor_objective); a seeded sample of blocks is solved again by the CPU
-oracle and compared block by block (identical masks, or a near-tie), and its
-exact optimum gives the quality gap, which must stay inside the pages' stated
-1-10% relative error.
+(tsenor_objective); a seeded sample of at least 2048 blocks is solved again by
+the CPU oracle and compared block by block: at least 99.9% of the sampled
+blocks identical, every differing one through a near-tie of the oracle's keys
+(relative gap below 1e-6), the summed objective within 1e-6 relative.  The
+sample's exact optimum gives the quality gap, which must stay inside the
+pages' stated 1-10% relative error.
 """
 import numpy as np
 import pytest
@@ -25,7 +27,7 @@ def gather_blocks(W, M, ids):
                           axis=1)
 
 
-def check_sampled(name, stor, W, dtype, N, M, tau, iters, sweeps, n_sample, seed=0):
+def check_sampled(name, stor, W, dtype, N, M, tau, iters, sweeps, n_sample, seed=0, min_identical=0.999):
     rows, cols = W.shape
     Wd = to_device(stor, dtype)
     tsl.tsenor_error_count()
@@ -55,15 +57,16 @@ def check_sampled(name, stor, W, dtype, N, M, tau, iters, sweeps, n_sample, seed
              "max_inverted_key_gap": max(gaps) if gaps else 0.0, "objective_rel": float(rel),
              "gap_mean": float(gap.mean()), "gap_max": float(gap.max())}
     record(name, stats)
+    assert same.mean() >= min_identical, stats
     assert all(g <= NEAR_TIE for g in gaps), stats
     assert rel <= 1e-6, stats
     assert (gap >= -1e-12).all() and gap.mean() <= 0.10, stats
     return stats
 
 
-@pytest.mark.parametrize("name,n_sample", [("w4096x4096_bf16_normal_8of16", 256),
-                                           ("w4096x11008_bf16_t3_16of32", 96),
-                                           ("w8192x28672_bf16_laplace_32of64", 24)])
+@pytest.mark.parametrize("name,n_sample", [("w4096x4096_bf16_normal_8of16", 4096),
+                                           ("w4096x11008_bf16_t3_16of32", 4096),
+                                           ("w8192x28672_bf16_laplace_32of64", 4096)])
 def test_full_workload_sampled(name, n_sample):
     w = synth.WORKLOADS[name]
     stor, W = synth.workload_matrix(w)
@@ -74,4 +77,4 @@ def test_stack_7b_layer_sampled():
     s = synth.STACK_7B_SETTINGS
     for k, (name, stor, W) in enumerate(synth.stack_7b_layer(0)):
         check_sampled(f"stack7b_layer0_{name}", stor, W, "bf16", s["N"], s["M"], s["tau"], s["iters"],
-                      s["sweeps"], 128, seed=k)
+                      s["sweeps"], 2048, seed=k)

@@ -1,5 +1,11 @@
-"""CPU checks of the algebraic forms the rounding kernels use in place of the
-pages' definitions (2-in/1-out local search, "What carries the argument"):
+"""CPU checks of the algebraic and floating-point forms the kernels use in
+place of the pages' definitions.  Dykstra ("What carries the argument"):
+
+  - the anchor points rebuild the linear-form exponentials as a product of
+    fp32 factors, which keeps a few ulps where the fp32 sum of the exponent's
+    terms does not (below).
+
+Rounding (2-in/1-out local search, "What carries the argument"):
 
   - pair gains in max-plus form: with C_x[j] = a_xj off row x's support
     (-inf on it) and Bn_x[j] = a_xj on it (+inf off it),
@@ -111,3 +117,48 @@ def test_every_row_has_a_partner_with_another_support(M, N):
         mask = random_valid_mask(M, N, rng)
         for x in range(M):
             assert any((mask[x] != mask[y]).any() for y in range(M) if y != x)
+
+
+# --- the anchor points of the kernels' linear-form exponentials --------------
+# The kernels rebuild E = 2^(y0 + U_i + V_j) every 64 iterations.  The terms
+# y0 and U_i + V_j are each of size up to tau * log2(e) and cancel; as a
+# product, (E0_ij * 2^U_i) * 2^V_j with E0 = 2^y0 taken once from an fp64 y0,
+# every entry carries a few fp32 roundings whatever the size of the terms.
+# These checks emulate both forms in numpy (fp32 roundings explicit, the
+# hardware exponential replaced by the correctly rounded one) against exact
+# fp64 values.
+
+def _exp2_wide(y):
+    """fp32 2^y for fp64 y in [-126, 126]: y = n + f, n the nearest integer, the
+    fp32 2^f scaled by the exact 2^n (the kernels' split)."""
+    y = np.clip(np.asarray(y, np.float64), -126.0, 126.0)
+    n = np.rint(y)
+    f = (y - n).astype(np.float32)
+    return (np.exp2(f.astype(np.float64)).astype(np.float32) * np.exp2(n).astype(np.float32)).astype(np.float32)
+
+
+def test_exp2_split_is_within_two_roundings():
+    rng = np.random.default_rng(0)
+    y = np.concatenate([rng.uniform(-60.0, 60.0, 20000), rng.uniform(-0.5, 0.5, 2000), [-43.28, 0.0, 17.5]])
+    got = _exp2_wide(y).astype(np.float64)
+    rel = np.abs(got / np.exp2(y) - 1.0)
+    assert rel.max() <= 2.0 ** -23          # f rounded (<= 2^-26 in the exponent) + one fp32 rounding
+
+
+def test_product_anchor_keeps_a_few_ulps_where_the_fp32_sum_does_not():
+    rng = np.random.default_rng(1)
+    tau2 = 30.0 * 1.4426950408889634
+    q = rng.uniform(0.0, 1.0, 50000)                # a / max|W|
+    y0 = tau2 * q - tau2                            # in [-tau2, 0], fp64
+    U = rng.uniform(0.0, tau2, q.size)              # row potentials of weak rows: large
+    V = rng.uniform(-2.0, 2.0, q.size)
+    exact = np.exp2(y0 + U + V)
+    E0 = _exp2_wide(y0)
+    prod = ((E0 * _exp2_wide(U)).astype(np.float32) * _exp2_wide(V)).astype(np.float32)
+    rel_prod = np.abs(prod.astype(np.float64) / exact - 1.0)
+    # fp32 sum of the terms, then the exponential (the form kept for very large tau)
+    s = (y0.astype(np.float32) + (U.astype(np.float32) + V.astype(np.float32))).astype(np.float32)
+    rel_sum = np.abs(np.exp2(s.astype(np.float64)) / exact - 1.0)
+    assert rel_prod.max() <= 5 * 2.0 ** -24       # E0, 2^U, 2^V and two products
+    assert rel_sum.max() >= 20 * 2.0 ** -24       # cancellation of terms of size ~tau2
+    assert np.median(rel_sum) > 4 * np.median(rel_prod)

@@ -191,3 +191,4 @@ def test_plan_bounds_at_finite_iterations():
     err = np.maximum(np.abs(B.sum(axis=3) - 2.0).max(axis=2), np.abs(B.sum(axis=2) - 2.0).max(axis=2))
     assert err.max() < 0.05
     assert np.median(err) < 1e-4
+
