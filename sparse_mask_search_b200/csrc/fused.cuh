@@ -8,7 +8,7 @@
 //  - M = 64: one CTA of 4 warps per block; the CTA sorts, warp 0 runs the
 //    greedy and the repair, all 128 threads the local search.
 // EXT instances add the warm start, the stop rule and the potentials export
-// of dykstra_tile_solve.  M = 16 and 64 stage the W tiles by TMA.
+// of dykstra_tile_solve.  M = 16, 32 and 64 stage the W tiles by TMA.
 #pragma once
 
 #include <type_traits>
@@ -21,21 +21,26 @@ namespace tsenor {
 
 // bf16: registers capped at 96, five CTAs per SM (shared memory would admit
 // six): 4.01 ms against 4.06 ms with the 80-register cap of six CTAs on the
-// 4096x11008 16:32 workload.  The fp32 key needs more registers.
-// The tile is read with 16-byte loads here, not staged by TMA: on the same
-// workload the TMA-staged variant of this kernel timed 5.16 ms against
-// 5.01 ms with the earlier exponential-per-iteration solver (the plan kernel
-// of the same M gained 0.7% from TMA staging).
+// 4096x11008 16:32 workload (an earlier solver); at the cap of four CTAs (128
+// registers, no spill) the current kernel takes 3.60 ms against 3.57.  The
+// fp32 key needs more registers.
+// W tiles are staged by TMA into the block's rounding space (free during the
+// solve), with the mbarrier in its row-count array.  A/B on the same workload
+// against 16-byte loads by the block's threads: 3.488 / 3.495 ms against
+// 3.490 ms (2.750 against 2.766 ms without the local search); with both paths
+// compiled into one kernel either one took about 3.56 ms.
 template <typename T, bool EXT = false>
 __global__ void __launch_bounds__(128, std::is_same<T, BF16>::value ? 5 : 4)
-fused_kernel32(const typename T::storage* __restrict__ W, int64_t cols, int64_t n_blocks, int N, float tau,
-               int iters, int sweeps, uint32_t* __restrict__ mask, int64_t wpr, DykstraExt ext = {}) {
+fused_kernel32(const __grid_constant__ CUtensorMap wmap, int64_t cols, int64_t n_blocks, int N, float tau, int iters,
+               int sweeps, uint32_t* __restrict__ mask, int64_t wpr, DykstraExt ext = {}) {
     constexpr int M = 32;
     using C = TileCfg<M>;
     using Key = typename KeyOf<T>::type;
     static_assert(C::TPB == 32 && C::BPC == 4, "one warp per block");
     constexpr int TS = M + 1;                       // tile row stride (conflict-free column access)
-    extern __shared__ __align__(16) unsigned char fused32_raw[];
+    static_assert((C::BPC * M * TS * 4) % 128 == 0 && sizeof(RoundShared<M>) % 128 == 0, "TMA staging alignment");
+    static_assert(sizeof(RoundShared<M>::G) >= M * M * sizeof(typename T::storage), "TMA staging size");
+    extern __shared__ __align__(128) unsigned char fused32_raw[];
     const TileThread<M> th;
     float* tile = reinterpret_cast<float*>(fused32_raw) + th.blk * M * TS;
     RoundShared<M>* shs = reinterpret_cast<RoundShared<M>*>(reinterpret_cast<float*>(fused32_raw) + C::BPC * M * TS);
@@ -45,10 +50,16 @@ fused_kernel32(const typename T::storage* __restrict__ W, int64_t cols, int64_t 
     const int64_t r0 = active ? (b / nbc) * M : 0, c0 = active ? (b % nbc) * M : 0;
 
     float S[C::P][C::Q];                      // plan of this thread's entries
-    const TileSource<T> src{nullptr, nullptr, nullptr, W, cols};
+    const TileSource<T> src{&wmap, reinterpret_cast<typename T::storage*>(shs[th.blk].G),
+                            reinterpret_cast<uint64_t*>(shs[th.blk].rc), nullptr, 0};
     const bool finite = dykstra_tile_solve<M, T, TS, EXT>(src, r0, c0, active, N, tau, iters, tile, nullptr, th, S,
                                                           ext, b);
     if (!active) return;                              // no CTA-wide barrier follows
+    // the tile's copy has landed and every lane has waited for it: the barrier's
+    // row-count slots are handed back to the rounding (a block whose copy did not
+    // land is failed and never rounded)
+    if (finite && th.lane == 0) mbar_inval(reinterpret_cast<uint64_t*>(shs[th.blk].rc));
+    __syncwarp();
 
     Key key[C::P * C::Q];
 #pragma unroll

@@ -152,11 +152,13 @@ cudaError_t launch_fused(const void* W, int64_t rows, int64_t cols, int N, float
         fused_kernel_small<M, T, EXT><<<dim3(unsigned((nb + bpc - 1) / bpc)), FusedSmallCfg<M>::THREADS, smem, st>>>(
             static_cast<const typename T::storage*>(W), cols, nb, N, tau, iters, sweeps, mask, wpr, ext);
     } else if constexpr (M == 32) {
-        const auto* w = static_cast<const typename T::storage*>(W);
+        CUtensorMap map;
+        e = encode_w_map<T>(&map, W, rows, cols, M);
+        if (e != cudaSuccess) return e;
         constexpr size_t smem = fused32_smem();
         e = cudaFuncSetAttribute(fused_kernel32<T, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
-        fused_kernel32<T, EXT><<<dim3(unsigned((nb + 3) / 4)), 128, smem, st>>>(w, cols, nb, N, tau, iters, sweeps,
+        fused_kernel32<T, EXT><<<dim3(unsigned((nb + 3) / 4)), 128, smem, st>>>(map, cols, nb, N, tau, iters, sweeps,
                                                                                mask, wpr, ext);
     } else if constexpr (M == 16) {
         CUtensorMap w;
