@@ -236,13 +236,22 @@ __device__ void cta_bitonic_sort64(Key (&key)[32], Key* xbuf, int warp, int lane
     }
 }
 
+// Integer image of a float that orders like the float (no NaN): the sign
+// bit flips the order of the negative half.  -0 is first made +0 (x + 0 in
+// round-to-nearest), so that the two zeros stay equal as in a float compare.
+__device__ __forceinline__ int ordered_bits(float f) {
+    const int b = __float_as_int(f + 0.f);
+    return b >= 0 ? b : b ^ 0x7fffffff;
+}
+__device__ __forceinline__ float from_ordered_bits(int k) { return __int_as_float(k >= 0 ? k : k ^ 0x7fffffff); }
+
+// Warp-wide (largest v, lowest i among the lanes holding it), returned to
+// every lane: two warp reductions (redux.sync) instead of a shuffle butterfly.
 __device__ __forceinline__ void warp_argmax(float& v, int& i) {
-#pragma unroll
-    for (int s = 16; s >= 1; s >>= 1) {
-        const float ov = __shfl_xor_sync(kFullMask, v, s);
-        const int oi = __shfl_xor_sync(kFullMask, i, s);
-        if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
-    }
+    const int k = ordered_bits(v);
+    const int km = __reduce_max_sync(kFullMask, k);
+    i = static_cast<int>(__reduce_min_sync(kFullMask, k == km ? static_cast<unsigned>(i) : 0xffffffffu));
+    v = from_ordered_bits(km);
 }
 
 // Sorted keys of one warp into sh.order.
@@ -561,11 +570,20 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
                 if (y != i && y != bp) { sh.G[bp * GS + y] = gb; sh.G[y * GS + bp] = gb; }
             }
             ls_barrier<NT>();                        // gain table and rows complete
-            if (row_thread) {
-                const int op = sh.bestp[y];
-                if (y == i || y == bp || op == i || op == bp) {
-                    rescan_row<M>(sh, y);
-                } else {
+            {
+                // rows i and bp, and rows whose best partner was one of them, are
+                // rescanned: for M = 32 by the whole warp, one row at a time (a
+                // warp argmax over the row's cached gains: lowest partner on ties,
+                // the diagonal is -inf), for M = 16 each by its own lane (a row of
+                // 16 gains); every other row compares its best with its new
+                // g(i, y), g(bp, y).  A/B: 16:32 3.499 -> 3.444 ms per call with
+                // the warp rescans, 8:16 1.125 -> 1.139 (so M = 16 keeps its own)
+                const int op = row_thread ? sh.bestp[y] : 0;
+                const bool need = row_thread && (y == i || y == bp || op == i || op == bp);
+                if constexpr (M < 32) {
+                    if (need) rescan_row<M>(sh, y);
+                }
+                if (row_thread && !need) {
                     float bv = sh.bestv[y];
                     int b2 = op;
                     const int c1 = i < bp ? i : bp, c2 = i < bp ? bp : i;
@@ -574,6 +592,18 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
                     if (g2 > bv || (g2 == bv && c2 < b2)) { bv = g2; b2 = c2; }
                     sh.bestv[y] = bv;
                     sh.bestp[y] = b2;
+                }
+                unsigned rows = M < 32 ? 0u : __ballot_sync(kFullMask, need);
+                while (rows) {
+                    const int x = __ffs(static_cast<int>(rows)) - 1;
+                    rows &= rows - 1;
+                    float g = lane < M ? sh.G[x * GS + lane] : -INFINITY;
+                    int p = lane;
+                    warp_argmax(g, p);
+                    if (lane == 0) {
+                        sh.bestv[x] = g;
+                        sh.bestp[x] = p;
+                    }
                 }
             }
             ls_barrier<NT>();                        // row bests complete
@@ -867,18 +897,39 @@ __device__ void local_search_mp(const float* a, float* Bm, float* Cm, const Roun
                 if (y != i && y != bp) { sh.G[bp * GS + y] = gb; sh.G[y * GS + bp] = gb; }
             }
             __syncthreads();                         // gain table and rows complete
-            const int op = sh.bestp[y];
-            if (y == i || y == bp || op == i || op == bp) {   // same for both threads of row y
-                rescan_row_pair<M>(sh, y, h, lane);
-            } else if (h == 0) {
-                float bv = sh.bestv[y];
-                int b2 = op;
-                const int c1 = i < bp ? i : bp, c2 = i < bp ? bp : i;
-                const float g1 = c1 == i ? gi : gb, g2 = c2 == i ? gi : gb;
-                if (g1 > bv || (g1 == bv && c1 < b2)) { bv = g1; b2 = c1; }
-                if (g2 > bv || (g2 == bv && c2 < b2)) { bv = g2; b2 = c2; }
-                sh.bestv[y] = bv;
-                sh.bestp[y] = b2;
+            {
+                // rows i and bp, and rows whose best partner was one of them: each
+                // warp rescans those of its 16 rows one at a time (a warp argmax
+                // over the row's 64 cached gains, lowest partner on ties; the
+                // diagonal, which holds no gain, is skipped); every other row
+                // compares its best with its new g(i, y), g(bp, y)
+                const int op = sh.bestp[y];
+                const bool need = y == i || y == bp || op == i || op == bp;   // same for both threads of row y
+                if (!need && h == 0) {
+                    float bv = sh.bestv[y];
+                    int b2 = op;
+                    const int c1 = i < bp ? i : bp, c2 = i < bp ? bp : i;
+                    const float g1 = c1 == i ? gi : gb, g2 = c2 == i ? gi : gb;
+                    if (g1 > bv || (g1 == bv && c1 < b2)) { bv = g1; b2 = c1; }
+                    if (g2 > bv || (g2 == bv && c2 < b2)) { bv = g2; b2 = c2; }
+                    sh.bestv[y] = bv;
+                    sh.bestp[y] = b2;
+                }
+                unsigned rows = __ballot_sync(kFullMask, need && h == 0);   // bit 2k: row 16 * warp + k
+                while (rows) {
+                    const int x = (tid >> 5) * 16 + (__ffs(static_cast<int>(rows)) - 1) / 2;
+                    rows &= rows - 1;
+                    const float g0 = lane == x ? -INFINITY : sh.G[x * GS + lane];
+                    const float g1 = lane + 32 == x ? -INFINITY : sh.G[x * GS + lane + 32];
+                    const bool hi = g1 > g0;                  // lower column on ties
+                    float g = hi ? g1 : g0;
+                    int p = (hi ? lane + 32 : lane) == x ? 0x7fff : (hi ? lane + 32 : lane);
+                    warp_argmax(g, p);
+                    if (lane == 0) {
+                        sh.bestv[x] = g;
+                        sh.bestp[x] = p;
+                    }
+                }
             }
             __syncthreads();                         // row bests complete
         }
