@@ -29,6 +29,7 @@
 #pragma once
 
 #include <climits>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -611,6 +612,148 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
     }
 }
 
+// ---------------------------------------------------------------------------
+// Sorting on 32-bit keys (bf16 inputs, blocks of E = M*M >= 256 entries).
+// The rounding order is (plan desc, |W| desc, flat index asc), a 64-bit key
+// (KeyB).  A 32-bit key orders all but a few entries the same way and halves
+// the work of every compare-exchange and shuffle:
+//   - clipped entries (plan exactly 1): (kOne + ((|W| bits + 1) << IB)) |
+//     (E-1-idx), above every other key and exact among themselves;
+//   - the others: the plan's bits with their IB lowest bits replaced by
+//     E-1-idx (IB = log2 E): exact wherever the plans differ above those bits.
+// After sorting on it, runs of adjacent entries that share the plan's upper
+// bits (near-ties, usually of two) are ordered by the full key with a few
+// passes of odd-even transposition; a block that has not settled after
+// kFixPasses passes (long runs of equal plans, as in a constant block) is
+// sorted again on the 64-bit keys.
+// ---------------------------------------------------------------------------
+struct Key32 {
+    unsigned k;
+    __device__ __forceinline__ bool before(const Key32& o) const { return k > o.k; }
+    __device__ __forceinline__ Key32 shfl_xor(int m) const { return Key32{__shfl_xor_sync(kFullMask, k, m)}; }
+};
+
+template <int E>
+struct Key32Fmt {
+    static constexpr int IB = E == 256 ? 8 : E == 1024 ? 10 : 12;
+    static_assert((1 << IB) == E, "E = 256, 1024 or 4096");
+    static constexpr unsigned kIdx = E - 1;
+    static constexpr unsigned kOne = 0x3F800000u;   // bits of 1.0f
+    __device__ __forceinline__ static unsigned make(unsigned long long kb) {
+        const unsigned s = static_cast<unsigned>(kb >> 32);
+        const unsigned inv = static_cast<unsigned>(kb) & kIdx;                  // E-1-idx
+        return s >= kOne ? (kOne + (((static_cast<unsigned>(kb >> 16) & 0xffffu) + 1u) << IB)) | inv
+                         : ((s & ~kIdx) | inv);
+    }
+    __device__ __forceinline__ static int index(unsigned k) { return static_cast<int>(kIdx - (k & kIdx)); }
+};
+
+constexpr int kFixPasses = 8;
+
+// Adjacent sorted keys x (earlier) and y: true when the full key puts y first.
+// Only entries below 1 with the same upper plan bits can be out of order;
+// their full keys are compared out of line (rare, and it keeps the unrolled
+// passes short: the fused kernels' code competes for the instruction cache).
+// sbits: plan bits by flat index; a: |W| with row stride M+1.
+template <int M>
+__device__ __noinline__ bool fix_swap_full(unsigned x, unsigned y, const unsigned* sbits, const float* a) {
+    using F = Key32Fmt<M * M>;
+    const int ix = F::index(x), iy = F::index(y);
+    const unsigned long long kx = (static_cast<unsigned long long>(sbits[ix]) << 32) |
+                                  (__float_as_uint(a[(ix / M) * (M + 1) + ix % M]) & 0xffff0000u) |
+                                  (0xffffu - static_cast<unsigned>(ix));
+    const unsigned long long ky = (static_cast<unsigned long long>(sbits[iy]) << 32) |
+                                  (__float_as_uint(a[(iy / M) * (M + 1) + iy % M]) & 0xffff0000u) |
+                                  (0xffffu - static_cast<unsigned>(iy));
+    return ky > kx;
+}
+template <int M>
+__device__ __forceinline__ bool fix_swap(unsigned x, unsigned y, const unsigned* sbits, const float* a) {
+    using F = Key32Fmt<M * M>;
+    if (x > F::kOne || ((x ^ y) & ~F::kIdx)) return false;
+    return fix_swap_full<M>(x, y, sbits, a);
+}
+
+// Odd-even transposition over the warp's sorted keys (position lane*R + r)
+// with the full key; returns whether a full pass made no exchange.
+template <int M, int R>
+__device__ bool fix_near_ties(Key32 (&k)[R], const unsigned* sbits, const float* a, int lane) {
+    static_assert(R % 2 == 0, "pairs (2m, 2m+1) within a lane");
+#pragma unroll 1
+    for (int pass = 0; pass < kFixPasses; ++pass) {
+        bool moved = false;
+#pragma unroll
+        for (int r = 0; r < R; r += 2)
+            if (fix_swap<M>(k[r].k, k[r + 1].k, sbits, a)) { const Key32 t = k[r]; k[r] = k[r + 1]; k[r + 1] = t; moved = true; }
+#pragma unroll
+        for (int r = 1; r + 1 < R; r += 2)
+            if (fix_swap<M>(k[r].k, k[r + 1].k, sbits, a)) { const Key32 t = k[r]; k[r] = k[r + 1]; k[r + 1] = t; moved = true; }
+        // the pair across the lane boundary: both lanes take the same decision
+        const unsigned nxt = __shfl_down_sync(kFullMask, k[0].k, 1);
+        const unsigned prv = __shfl_up_sync(kFullMask, k[R - 1].k, 1);
+        const bool down = lane < 31 && fix_swap<M>(k[R - 1].k, nxt, sbits, a);
+        const bool up = lane > 0 && fix_swap<M>(prv, k[0].k, sbits, a);
+        if (down) k[R - 1].k = nxt;
+        if (up) k[0].k = prv;
+        moved = moved || down || up;
+        if (!__any_sync(kFullMask, moved)) return true;
+    }
+    return false;
+}
+
+// The 64-bit sort of a block whose 32-bit keys did not settle, from the plan
+// bits (sbits, by flat index), |W| and the index: out of line, so that this
+// rarely taken path does not enlarge the fused kernels' loops (the
+// instruction cache of an SM holds the code of warps in every phase).
+template <int M>
+__device__ __noinline__ void sort_to_order_full(const unsigned* sbits, const float* a, const RoundView<M>& sh,
+                                                int lane) {
+    constexpr int R = WarpRound<M>::R;
+    KeyB kb[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int e = lane * R + r;                  // any assignment of entries to positions
+        kb[r] = KeyB::make(__uint_as_float(sbits[e]), a[(e / M) * (M + 1) + e % M], e);
+    }
+    warp_bitonic_sort<R>(kb, lane);
+    __syncwarp();                                    // sbits read by every lane before the order overlays it
+    keys_to_order<M>(kb, sh, lane);
+}
+
+// Step 1 for bf16 keys: sort on Key32, settle the near-ties, write the order;
+// a block that does not settle is sorted on its 64-bit keys.  sbits: E words
+// of shared memory that the order does not need until this returns (the gain
+// table's space).
+template <int M>
+__device__ void sort_to_order(KeyB (&key)[WarpRound<M>::R], const float* a, const RoundView<M>& sh,
+                              unsigned* sbits, int lane) {
+    constexpr int R = WarpRound<M>::R, E = M * M;
+    using F = Key32Fmt<E>;
+    static_assert(E % 32 == 0 && E >= 256, "no padding keys");
+    Key32 k[R];
+    bool above_one = false;                          // a given plan above 1: only the 64-bit keys order it
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const unsigned sb = static_cast<unsigned>(key[r].k >> 32);
+        sbits[key[r].index()] = sb;
+        above_one = above_one || sb > F::kOne;
+        k[r] = Key32{F::make(key[r].k)};
+    }
+    __syncwarp();
+    bool fast = !__any_sync(kFullMask, above_one);
+    if (fast) {
+        warp_bitonic_sort<R>(k, lane);
+        fast = fix_near_ties<M, R>(k, sbits, a, lane);
+    }
+    if (fast) {
+        __syncwarp();                                // sbits read by every lane before the order overlays it
+#pragma unroll
+        for (int r = 0; r < R; ++r) sh.order[lane * R + r] = static_cast<uint16_t>(F::index(k[r].k));
+    } else {
+        sort_to_order_full<M>(sbits, a, sh, lane);
+    }
+}
+
 // Steps 1-4 for one block (M <= 32).  `key` holds this lane's keys (any
 // assignment of the block's entries to positions; padding positions hold
 // Key::sentinel()), `a` the block's |W| (row stride M+1, shared memory).
@@ -620,8 +763,12 @@ template <int M, typename Key>
 __device__ bool round_block_warp(Key (&key)[WarpRound<M>::R], const float* a, const RoundView<M>& sh, int N,
                                  int sweeps, int lane) {
     constexpr int R = WarpRound<M>::R;
-    warp_bitonic_sort<R>(key, lane);
-    keys_to_order<M>(key, sh, lane);
+    if constexpr (std::is_same<Key, KeyB>::value && M >= 16) {
+        sort_to_order<M>(key, a, sh, reinterpret_cast<unsigned*>(sh.G), lane);
+    } else {
+        warp_bitonic_sort<R>(key, lane);
+        keys_to_order<M>(key, sh, lane);
+    }
     __syncwarp();
     if (!greedy_and_repair<M, WarpRound<M>::EP>(a, sh, N, lane)) return false;
     if (sweeps <= 0) return true;
@@ -973,6 +1120,9 @@ __device__ bool round_block_cta64(Key (&key)[32], Round64Smem<Key>& sm, int N, i
     constexpr int M = 64;
     const int lane = tid & 31, warp = tid >> 5;
     const RoundView<M> sh = sm.view();
+    // the 64-bit keys: with 4096 entries the 32-bit keys of sort_to_order drop
+    // 12 plan bits, and the near-ties they leave made this sort slower (A/B:
+    // 35.00 -> 35.42 ms per 32:64 call)
     cta_bitonic_sort64(key, sm.u.xbuf, warp, lane);
     __syncthreads();
 #pragma unroll

@@ -162,3 +162,78 @@ def test_product_anchor_keeps_a_few_ulps_where_the_fp32_sum_does_not():
     assert rel_prod.max() <= 5 * 2.0 ** -24       # E0, 2^U, 2^V and two products
     assert rel_sum.max() >= 20 * 2.0 ** -24       # cancellation of terms of size ~tau2
     assert np.median(rel_sum) > 4 * np.median(rel_prod)
+
+
+# --- the rounding sort's 32-bit keys (bf16 inputs, blocks of 256 and 1024) ---
+# The kernels sort on a 32-bit image of the rounding key (plan desc, |W| desc,
+# flat index asc): clipped entries (plan exactly 1) as (1.0f bits +
+# ((|W| bits + 1) << IB)) | (E-1-idx), the others as the plan's bits with their
+# IB low bits replaced by E-1-idx; then odd-even transposition passes with the
+# full key settle runs that share the plan's upper bits; a block not settled
+# after 8 passes, or holding a plan above 1, is sorted on the full key.
+
+def _full_key(S, a, idx):
+    return ((S.view(np.uint32).astype(np.uint64) << np.uint64(32))
+            | (a.view(np.uint32).astype(np.uint64) & np.uint64(0xffff0000))
+            | (np.uint64(0xffff) - idx.astype(np.uint64)))
+
+
+def _key32(kb, E):
+    IB = E.bit_length() - 1
+    s = (kb >> np.uint64(32)) & np.uint64(0xffffffff)
+    inv = kb & np.uint64(E - 1)
+    a16 = (kb >> np.uint64(16)) & np.uint64(0xffff)
+    one = np.uint64(0x3F800000)
+    return np.where(s >= one, (one + ((a16 + np.uint64(1)) << np.uint64(IB))) | inv,
+                    (s & ~np.uint64(E - 1)) | inv)
+
+
+def _sort32_then_settle(S, a, E, passes=8):
+    """The kernels' order by the 32-bit keys and the settling passes; None = not settled."""
+    kb = _full_key(S, a, np.arange(E))
+    k = sorted((int(v) for v in _key32(kb, E)), reverse=True)
+    full = [int(v) for v in kb]
+    idx = lambda x: (E - 1) - (x & (E - 1))
+
+    def later_first(x, y):
+        if x > 0x3F800000 or ((x ^ y) & ~(E - 1)):
+            return False
+        return full[idx(y)] > full[idx(x)]
+    for _ in range(passes):
+        moved = False
+        for start in (0, 1):
+            for q in range(start, E - 1, 2):
+                if later_first(k[q], k[q + 1]):
+                    k[q], k[q + 1] = k[q + 1], k[q]
+                    moved = True
+        if not moved:
+            return [idx(v) for v in k]
+    return None
+
+
+@pytest.mark.parametrize("E", [256, 1024])
+def test_32bit_sort_keys_give_the_rounding_order(E):
+    rng = np.random.default_rng(E)
+    settled = 0
+    for t in range(12):
+        S = rng.random(E).astype(np.float32)
+        if t % 3 == 0:
+            S[rng.random(E) < 0.3] = 1.0                     # clipped entries
+        if t % 2 == 1:
+            S = (np.round(S * 500) / 500).astype(np.float32)  # many equal and near-equal plans
+        a = (np.abs(rng.standard_normal(E)).astype(np.float32).view(np.uint32) & 0xffff0000).view(np.float32)
+        if t % 4 == 0:
+            a[rng.random(E) < 0.5] = 0.0                     # ties of |W|
+        kb = _full_key(S, a, np.arange(E))
+        truth = sorted(range(E), key=lambda i: -int(kb[i]))
+        got = _sort32_then_settle(S, a, E)
+        if got is not None:
+            settled += 1
+            assert got == truth
+    assert settled >= 1
+    # a constant block: the index decides, as in the 32-bit keys, and nothing moves
+    assert _sort32_then_settle(np.full(E, 0.5, np.float32), np.full(E, 1.0, np.float32), E) == list(range(E))
+    # equal plans with |W| rising along the index reverse the whole block: it does not
+    # settle in 8 passes, and the 64-bit sort takes it
+    ramp = ((np.arange(E, dtype=np.float32) + 1.0).view(np.uint32) & 0xffff0000).view(np.float32)
+    assert _sort32_then_settle(np.full(E, 0.5, np.float32), ramp, E) is None
