@@ -73,14 +73,6 @@ __device__ __forceinline__ float exp2_wide(double y) {
 }
 
 
-// E0 = 2^y0 of one entry, y0 = tau2 (a / max|W| - 1) in fp64.  Out of line:
-// inlined 64 times into the one-thread-per-block solver (M = 8) it made the
-// compiler keep many fp64 temporaries live at once and spill the solver's
-// registers; as a call it costs a few instructions per entry, once.
-__device__ __noinline__ float e0_of(double tau2d, float a, double inv_m) {
-    return exp2_wide(fma(tau2d, double(a) * inv_m, -tau2d));
-}
-
 // ---------------------------------------------------------------------------
 // M = 4, 8: one thread holds a whole block in registers.  Rows are streamed:
 // the exponentials of one row live only until its column contributions are
@@ -137,11 +129,14 @@ __device__ __forceinline__ bool dykstra_thread_solve(const typename T::storage* 
 #pragma unroll
     for (int i = 0; i < M; ++i) {
 #pragma unroll
-        for (int j = 0; j < M; ++j) y[i][j] = e0_of(tau2d, y[i][j], inv_m);
+        for (int j = 0; j < M; ++j) y[i][j] = exp2_wide(fma(tau2d, double(y[i][j]) * inv_m, -tau2d));
 #pragma unroll
         for (int v = 0; v < M / 4; ++v)
             reinterpret_cast<float4*>(y0s + i * M)[v] = make_float4(y[i][4 * v], y[i][4 * v + 1], y[i][4 * v + 2],
                                                                     y[i][4 * v + 3]);
+        // one row's fp64 temporaries at a time: with the rows interleaved the
+        // compiler kept many of them live and spilled the solver's registers
+        asm volatile("" ::: "memory");
     }
     const float fN = float(N);
 
