@@ -616,16 +616,23 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
 // Sorting on 32-bit keys (bf16 inputs, blocks of E = M*M >= 256 entries).
 // The rounding order is (plan desc, |W| desc, flat index asc), a 64-bit key
 // (KeyB).  A 32-bit key orders all but a few entries the same way and halves
-// the work of every compare-exchange and shuffle:
-//   - clipped entries (plan exactly 1): (kOne + ((|W| bits + 1) << IB)) |
-//     (E-1-idx), above every other key and exact among themselves;
-//   - the others: the plan's bits with their IB lowest bits replaced by
-//     E-1-idx (IB = log2 E): exact wherever the plans differ above those bits.
-// After sorting on it, runs of adjacent entries that share the plan's upper
-// bits (near-ties, usually of two) are ordered by the full key with a few
-// passes of odd-even transposition; a block that has not settled after
-// kFixPasses passes (long runs of equal plans, as in a constant block) is
-// sorted again on the 64-bit keys.
+// the work of every compare-exchange and shuffle.  Its IB = log2 E low bits
+// hold E-1-idx, the 32-IB bits above them a bucket of the plan:
+//   - plan exactly 1 (clipped): nibble 15, then the |W| bits: exact among
+//     the clipped entries and above every other bucket;
+//   - plan in [2^-14, 1): nibble e-112 (e the biased exponent, 113..126),
+//     then the MB = 28-IB upper mantissa bits;
+//   - plan below 2^-14: nibble 0, then the plan's bits shifted right so that
+//     they fit the MB bits (monotone, coarse).
+// The 4-bit exponent window spends the key's bits on the binades the plans
+// occupy (on the synthetic 32:64 workload, tau = 30, every plan lies in
+// [2^-8, 1]), so that 4096-entry blocks keep 16 mantissa bits (A/B against
+// the plan's upper bits without the window, 4096x11008 16:32 workload: 3.413
+// -> 3.289 ms per call).  After sorting on it, runs of
+// adjacent entries in the same bucket (near-ties, usually of two) are ordered
+// by the full key with a few passes of odd-even transposition; a block that
+// has not settled after kFixPasses passes (long runs of equal plans, as in a
+// constant block) is sorted again on the 64-bit keys.
 // ---------------------------------------------------------------------------
 struct Key32 {
     unsigned k;
@@ -637,21 +644,28 @@ template <int E>
 struct Key32Fmt {
     static constexpr int IB = E == 256 ? 8 : E == 1024 ? 10 : 12;
     static_assert((1 << IB) == E, "E = 256, 1024 or 4096");
+    static constexpr int MB = 28 - IB;                // mantissa bits of a bucket
     static constexpr unsigned kIdx = E - 1;
-    static constexpr unsigned kOne = 0x3F800000u;   // bits of 1.0f
+    static constexpr unsigned kOne = 0x3F800000u;     // bits of 1.0f
+    static constexpr unsigned kLowExp = 112;          // biased exponents up to this share nibble 0
     __device__ __forceinline__ static unsigned make(unsigned long long kb) {
         const unsigned s = static_cast<unsigned>(kb >> 32);
         const unsigned inv = static_cast<unsigned>(kb) & kIdx;                  // E-1-idx
-        return s >= kOne ? (kOne + (((static_cast<unsigned>(kb >> 16) & 0xffffu) + 1u) << IB)) | inv
-                         : ((s & ~kIdx) | inv);
+        const unsigned ex = s >> 23;
+        const unsigned bucket =
+            s >= kOne ? ((15u << MB) | (static_cast<unsigned>(kb >> 16) & 0xffffu))
+            : ex > kLowExp ? (((ex - kLowExp) << MB) | ((s >> (23 - MB)) & ((1u << MB) - 1u)))
+                           : (s >> (30 - MB));
+        return (bucket << IB) | inv;
     }
+    __device__ __forceinline__ static bool clipped(unsigned k) { return (k >> 28) == 15u; }
     __device__ __forceinline__ static int index(unsigned k) { return static_cast<int>(kIdx - (k & kIdx)); }
 };
 
 constexpr int kFixPasses = 8;
 
 // Adjacent sorted keys x (earlier) and y: true when the full key puts y first.
-// Only entries below 1 with the same upper plan bits can be out of order;
+// Only entries below 1 in the same bucket can be out of order;
 // their full keys are compared out of line (rare, and it keeps the unrolled
 // passes short: the fused kernels' code competes for the instruction cache).
 // sbits: plan bits by flat index; a: |W| with row stride M+1.
@@ -670,7 +684,7 @@ __device__ __noinline__ bool fix_swap_full(unsigned x, unsigned y, const unsigne
 template <int M>
 __device__ __forceinline__ bool fix_swap(unsigned x, unsigned y, const unsigned* sbits, const float* a) {
     using F = Key32Fmt<M * M>;
-    if (x > F::kOne || ((x ^ y) & ~F::kIdx)) return false;
+    if (F::clipped(x) || ((x ^ y) & ~F::kIdx)) return false;
     return fix_swap_full<M>(x, y, sbits, a);
 }
 
@@ -1106,11 +1120,104 @@ struct Round64Smem {
     } v;
     int ok;
     int xj[2];                                       // local search: the entries of the current swap
+    unsigned bnd[8];                                 // 32-bit sort: first and last key of each warp
     uint64_t tma_bar;                                // fused kernel: completion of the W tile copy
     __device__ __forceinline__ RoundView<64> view() {
         return RoundView<64>{a, u.gr.order, v.rb.rowbits, v.rb.bestv, v.rb.bestp, u.gr.rc, u.gr.cc, nullptr};
     }
 };
+
+// Odd-even transposition over the CTA's 4096 sorted 32-bit keys (position
+// t*32 + r, t = warp*32 + lane) with the full key, as fix_near_ties; the
+// pairs across warps go through sm.bnd.  Returns whether a full pass made
+// no exchange (uniform over the CTA).
+__device__ bool cta_fix_near_ties64(Key32 (&k)[32], const unsigned* sbits, const float* a, unsigned* bnd, int warp,
+                                    int lane) {
+    constexpr int R = 32, M = 64;
+#pragma unroll 1
+    for (int pass = 0; pass < kFixPasses; ++pass) {
+        bool moved = false;
+#pragma unroll
+        for (int r = 0; r < R; r += 2)
+            if (fix_swap<M>(k[r].k, k[r + 1].k, sbits, a)) { const Key32 t = k[r]; k[r] = k[r + 1]; k[r + 1] = t; moved = true; }
+#pragma unroll
+        for (int r = 1; r + 1 < R; r += 2)
+            if (fix_swap<M>(k[r].k, k[r + 1].k, sbits, a)) { const Key32 t = k[r]; k[r] = k[r + 1]; k[r + 1] = t; moved = true; }
+        unsigned nxt = __shfl_down_sync(kFullMask, k[0].k, 1);
+        unsigned prv = __shfl_up_sync(kFullMask, k[R - 1].k, 1);
+        if (lane == 0) bnd[warp] = k[0].k;
+        if (lane == 31) bnd[4 + warp] = k[R - 1].k;
+        __syncthreads();
+        if (lane == 31 && warp < 3) nxt = bnd[warp + 1];
+        if (lane == 0 && warp > 0) prv = bnd[4 + warp - 1];
+        // both threads of a pair take the same decision from the same two keys
+        const bool down = (lane < 31 || warp < 3) && fix_swap<M>(k[R - 1].k, nxt, sbits, a);
+        const bool up = (lane > 0 || warp > 0) && fix_swap<M>(prv, k[0].k, sbits, a);
+        if (down) k[R - 1].k = nxt;
+        if (up) k[0].k = prv;
+        moved = moved || down || up;
+        if (!__syncthreads_or(moved)) return true;   // also orders this pass's bnd reads before the next writes
+    }
+    return false;
+}
+
+// The 64-bit sort of an M = 64 block whose 32-bit keys did not settle (or
+// that holds a plan above 1), from the plan bits (sbits, by flat index) and
+// |W|; out of line, as sort_to_order_full.
+__device__ __noinline__ void cta_sort_to_order64_full(const unsigned* sbits, Round64Smem<KeyB>& sm, int warp,
+                                                      int lane) {
+    constexpr int M = 64, R = 32;
+    const int t = warp * 32 + lane;
+    KeyB kb[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int e = t * R + r;                     // any assignment of entries to positions
+        kb[r] = KeyB::make(__uint_as_float(sbits[e]), sm.a[(e / M) * (M + 1) + e % M], e);
+    }
+    __syncthreads();                                 // sbits read by all before the exchange space is reused
+    cta_bitonic_sort64(kb, sm.u.xbuf, warp, lane);
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < R; ++r) sm.u.gr.order[t * R + r] = static_cast<uint16_t>(kb[r].index());
+}
+
+// Step 1 for one M = 64 block of bf16 keys by the CTA: sort on Key32 (the
+// exchange buffer in the first 16 KB of the block's exchange space, the plan
+// bits by flat index in the second), settle the near-ties, write the order;
+// a block that does not settle is sorted on its 64-bit keys.  Every thread
+// calls it.  A/B against the 64-bit sort, 8192x28672 32:64 workload: 34.99 ->
+// 34.05 ms per call (a bucket of the plan's upper 20 bits, without the
+// exponent window, had left too many near-ties: 35.00 -> 35.42 ms).
+__device__ void cta_sort_to_order64(KeyB (&key)[32], Round64Smem<KeyB>& sm, int warp, int lane) {
+    constexpr int R = 32, E = 4096;
+    using F = Key32Fmt<E>;
+    static_assert(sizeof(sm.u) >= 2 * E * sizeof(unsigned), "exchange space: keys and plan bits");
+    static_assert(sizeof(uint16_t) * E + sizeof(int) * 128 <= sizeof(unsigned) * E, "the order stays clear of sbits");
+    Key32* xbuf = reinterpret_cast<Key32*>(&sm.u);
+    unsigned* sbits = reinterpret_cast<unsigned*>(&sm.u) + E;
+    const int t = warp * 32 + lane;
+    Key32 k[R];
+    bool above_one = false;                          // a given plan above 1: only the 64-bit keys order it
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const unsigned sb = static_cast<unsigned>(key[r].k >> 32);
+        sbits[key[r].index()] = sb;
+        above_one = above_one || sb > F::kOne;
+        k[r] = Key32{F::make(key[r].k)};
+    }
+    bool fast = !__syncthreads_or(above_one);        // also publishes sbits
+    if (fast) {
+        cta_bitonic_sort64(k, xbuf, warp, lane);     // ends with a barrier after its last exchange
+        fast = cta_fix_near_ties64(k, sbits, sm.a, sm.bnd, warp, lane);
+    }
+    if (fast) {
+        // the order overlays the key exchange buffer (no longer read), not sbits
+#pragma unroll
+        for (int r = 0; r < R; ++r) sm.u.gr.order[t * R + r] = static_cast<uint16_t>(F::index(k[r].k));
+    } else {
+        cta_sort_to_order64_full(sbits, sm, warp, lane);
+    }
+}
 
 // Steps 1-4 for one M = 64 block by a CTA of 4 warps (every thread calls it;
 // the result is uniform over the CTA).  `key`: this thread's 32 keys; sm.a:
@@ -1120,13 +1227,14 @@ __device__ bool round_block_cta64(Key (&key)[32], Round64Smem<Key>& sm, int N, i
     constexpr int M = 64;
     const int lane = tid & 31, warp = tid >> 5;
     const RoundView<M> sh = sm.view();
-    // the 64-bit keys: with 4096 entries the 32-bit keys of sort_to_order drop
-    // 12 plan bits, and the near-ties they leave made this sort slower (A/B:
-    // 35.00 -> 35.42 ms per 32:64 call)
-    cta_bitonic_sort64(key, sm.u.xbuf, warp, lane);
-    __syncthreads();
+    if constexpr (std::is_same<Key, KeyB>::value) {
+        cta_sort_to_order64(key, sm, warp, lane);
+    } else {
+        cta_bitonic_sort64(key, sm.u.xbuf, warp, lane);
+        __syncthreads();
 #pragma unroll
-    for (int r = 0; r < 32; ++r) sh.order[tid * 32 + r] = static_cast<uint16_t>(key[r].index());
+        for (int r = 0; r < 32; ++r) sh.order[tid * 32 + r] = static_cast<uint16_t>(key[r].index());
+    }
     __syncthreads();
     if (warp == 0) {
         const bool g = greedy_and_repair<M, 4096>(sm.a, sh, N, lane);

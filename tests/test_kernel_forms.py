@@ -164,13 +164,15 @@ def test_product_anchor_keeps_a_few_ulps_where_the_fp32_sum_does_not():
     assert np.median(rel_sum) > 4 * np.median(rel_prod)
 
 
-# --- the rounding sort's 32-bit keys (bf16 inputs, blocks of 256 and 1024) ---
+# --- the rounding sort's 32-bit keys (bf16 inputs, blocks of 256, 1024, 4096) ---
 # The kernels sort on a 32-bit image of the rounding key (plan desc, |W| desc,
-# flat index asc): clipped entries (plan exactly 1) as (1.0f bits +
-# ((|W| bits + 1) << IB)) | (E-1-idx), the others as the plan's bits with their
-# IB low bits replaced by E-1-idx; then odd-even transposition passes with the
-# full key settle runs that share the plan's upper bits; a block not settled
-# after 8 passes, or holding a plan above 1, is sorted on the full key.
+# flat index asc): the IB = log2 E low bits hold E-1-idx, the bits above them a
+# bucket of the plan - nibble 15 and the |W| bits for a plan of exactly 1,
+# nibble e-112 and the upper 28-IB mantissa bits for a plan in [2^-14, 1) (e
+# its biased exponent), nibble 0 and the plan's bits shifted right by 2+IB
+# below 2^-14; then odd-even transposition passes with the full key settle the
+# runs that share a bucket; a block not settled after 8 passes, or holding a
+# plan above 1, is sorted on the full key.
 
 def _full_key(S, a, idx):
     return ((S.view(np.uint32).astype(np.uint64) << np.uint64(32))
@@ -180,12 +182,20 @@ def _full_key(S, a, idx):
 
 def _key32(kb, E):
     IB = E.bit_length() - 1
-    s = (kb >> np.uint64(32)) & np.uint64(0xffffffff)
-    inv = kb & np.uint64(E - 1)
-    a16 = (kb >> np.uint64(16)) & np.uint64(0xffff)
-    one = np.uint64(0x3F800000)
-    return np.where(s >= one, (one + ((a16 + np.uint64(1)) << np.uint64(IB))) | inv,
-                    (s & ~np.uint64(E - 1)) | inv)
+    MB = 28 - IB
+    u = np.uint64
+    s = (kb >> u(32)) & u(0xffffffff)
+    inv = kb & u(E - 1)
+    a16 = (kb >> u(16)) & u(0xffff)
+    ex = s >> u(23)
+    bucket = np.where(s >= u(0x3F800000), (u(15) << u(MB)) | a16,
+                      np.where(ex > u(112), ((ex - np.minimum(ex, u(112))) << u(MB)) | ((s >> u(23 - MB)) & u((1 << MB) - 1)),
+                               s >> u(30 - MB)))
+    return (bucket << u(IB)) | inv
+
+
+def _clipped32(x):
+    return (x >> 28) == 15
 
 
 def _sort32_then_settle(S, a, E, passes=8):
@@ -196,7 +206,7 @@ def _sort32_then_settle(S, a, E, passes=8):
     idx = lambda x: (E - 1) - (x & (E - 1))
 
     def later_first(x, y):
-        if x > 0x3F800000 or ((x ^ y) & ~(E - 1)):
+        if _clipped32(x) or ((x ^ y) & ~(E - 1)):
             return False
         return full[idx(y)] > full[idx(x)]
     for _ in range(passes):
@@ -211,7 +221,7 @@ def _sort32_then_settle(S, a, E, passes=8):
     return None
 
 
-@pytest.mark.parametrize("E", [256, 1024])
+@pytest.mark.parametrize("E", [256, 1024, 4096])
 def test_32bit_sort_keys_give_the_rounding_order(E):
     rng = np.random.default_rng(E)
     settled = 0
@@ -237,3 +247,37 @@ def test_32bit_sort_keys_give_the_rounding_order(E):
     # settle in 8 passes, and the 64-bit sort takes it
     ramp = ((np.arange(E, dtype=np.float32) + 1.0).view(np.uint32) & 0xffff0000).view(np.float32)
     assert _sort32_then_settle(np.full(E, 0.5, np.float32), ramp, E) is None
+
+
+@pytest.mark.parametrize("E", [256, 1024, 4096])
+def test_32bit_key_buckets_are_monotone_in_the_full_key(E):
+    """A larger full key never gets a smaller bucket: so two keys can only be
+    out of order within a bucket, which is all the settling passes look at."""
+    rng = np.random.default_rng(7 + E)
+    n = 200000
+    # plans over every range the bucket treats apart: 1, the window's binades,
+    # below 2^-14 down to subnormals and 0, and the window's edges
+    S = np.concatenate([
+        np.ones(1000, np.float32),
+        rng.random(n // 2).astype(np.float32),
+        np.exp2(rng.uniform(-30, 0, n // 2)).astype(np.float32),
+        np.array([0.0, 1e-45, 2.0 ** -126, 2.0 ** -14, np.nextafter(np.float32(2.0 ** -14), np.float32(0)),
+                  np.nextafter(np.float32(1), np.float32(0)), 0.5], np.float32)])
+    a = (np.abs(rng.standard_normal(S.size)).astype(np.float32).view(np.uint32) & 0xffff0000).view(np.float32)
+    a[:50] = 0.0
+    idx = rng.integers(0, E, S.size)
+    kb = _full_key(S, a, idx)
+    k32 = _key32(kb, E)
+    order = np.argsort(kb, kind="stable")
+    b = (k32 >> np.uint64(E.bit_length() - 1))[order]
+    assert (np.diff(b.astype(np.int64)) >= 0).all()
+    # the clipped bucket sits above every other, and is exact among its own entries
+    clipped = S == 1.0
+    assert k32[clipped].min() > k32[~clipped].max()
+    assert _clipped32(int(k32[clipped][0])) and not _clipped32(int(k32[~clipped].max()))
+    # the window keeps 28 - log2 E mantissa bits: plans one step of that size apart differ
+    MB = 28 - (E.bit_length() - 1)
+    x = np.float32(0.3)
+    y = (x.view(np.uint32) + np.uint32(1 << (23 - MB))).view(np.float32)
+    kx, ky = _key32(_full_key(np.array([x, y]), np.zeros(2, np.float32), np.zeros(2, np.int64)), E)
+    assert (ky >> np.uint64(E.bit_length() - 1)) == (kx >> np.uint64(E.bit_length() - 1)) + np.uint64(1)
