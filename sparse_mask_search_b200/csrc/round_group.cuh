@@ -96,8 +96,8 @@ __device__ bool group_greedy_and_repair(const float* a, const RoundView<M>& sh, 
         }
         if ((acc >> lane) & 1u) atomicOr(&sh.rowbits[i], Bits(1) << j);
         const unsigned ga = mr & acc, gc = mc & acc;
-        if (ga && __ffs(ga) - 1 == lane) sh.rc[i] += __popc(ga);
-        if (gc && __ffs(gc) - 1 == lane) sh.cc[j] += __popc(gc);
+        if (ga && __ffs(ga) - 1 == lane) sh.rc[i] = r0c + __popc(ga);   // the counts read at the chunk's start
+        if (gc && __ffs(gc) - 1 == lane) sh.cc[j] = c0c + __popc(gc);
         taken += __popc(acc);
         __syncwarp(gmask);
     }

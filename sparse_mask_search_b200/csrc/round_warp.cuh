@@ -310,8 +310,8 @@ __device__ bool greedy_and_repair(const float* a, const RoundView<M>& sh, int N,
         // accepted lane of each row (column) group adds the group's count
         if (mine_acc) atomicOr(reinterpret_cast<unsigned*>(&sh.rowbits[i]) + (j >> 5), 1u << (j & 31));
         const unsigned ga = mr & acc, gc = mc & acc;
-        if (ga && __ffs(ga) - 1 == lane) sh.rc[i] += __popc(ga);
-        if (gc && __ffs(gc) - 1 == lane) sh.cc[j] += __popc(gc);
+        if (ga && __ffs(ga) - 1 == lane) sh.rc[i] = r0c + __popc(ga);   // the counts read at the chunk's start
+        if (gc && __ffs(gc) - 1 == lane) sh.cc[j] = c0c + __popc(gc);
         taken += __popc(acc);
         __syncwarp();
     }

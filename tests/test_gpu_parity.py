@@ -231,3 +231,28 @@ def test_mask_equals_rounding_of_exported_plan(c):
     m1 = tsl.tsenor_mask(Wd, N, M, tau, iters, sweeps)
     m2 = tsl.tsenor_round(tsl.tsenor_plan(Wd, N, M, tau, iters), Wd, N, M, sweeps)
     assert torch.equal(m1, m2)
+
+
+@pytest.mark.parametrize("M,N,rows,cols", [(16, 8, 128, 128), (32, 16, 128, 256), (64, 32, 256, 512)])
+def test_rounding_bit_exact_on_adversarial_keys(M, N, rows, cols):
+    """The bf16 sort's 32-bit keys keep a bucket of the plan (an exponent window
+    and upper mantissa bits) and settle same-bucket runs with the full key: keys
+    spread over many binades (below the window too), keys one or two ulps apart
+    (same bucket, any order), keys on bucket edges and exact ties of plan and
+    |W| must all round as the oracle does."""
+    g = np.random.default_rng(M * 31 + N)
+    stor, W = synth.make_matrix(rows, cols, "bf16", "laplace_outliers", 0.02, seed=77 + M)
+    Wd = to_device(stor, "bf16")
+    wide = np.exp2(g.uniform(-24.0, 0.0, (rows, cols))).astype(np.float32)
+    base = g.uniform(0.25, 0.5, (rows, cols)).astype(np.float32)
+    near = (base.view(np.uint32) & ~np.uint32(3) | g.integers(0, 4, (rows, cols)).astype(np.uint32)).view(np.float32)
+    edges = np.exp2(g.integers(-16, 1, (rows, cols)).astype(np.float32)) * \
+        np.where(g.random((rows, cols)) < 0.5, np.float32(1.0), np.float32(1.0 - 2.0 ** -24))
+    edges = np.minimum(edges, np.float32(1.0)).astype(np.float32)
+    few = (g.integers(0, 40, (rows, cols)) / 39.0).astype(np.float32)
+    for name, keys in (("wide", wide), ("near", near), ("edges", edges), ("few", few)):
+        kd = torch.from_numpy(keys).cuda()
+        m_gpu = mask_to_np(tsl.tsenor_round(kd, Wd, N, M, 8))
+        m_ref, st = oracle.round_plan(keys, W, N, M, 8)
+        assert st["failures"] == 0
+        assert (m_gpu == m_ref).all(), name
