@@ -281,3 +281,22 @@ def test_32bit_key_buckets_are_monotone_in_the_full_key(E):
     y = (x.view(np.uint32) + np.uint32(1 << (23 - MB))).view(np.float32)
     kx, ky = _key32(_full_key(np.array([x, y]), np.zeros(2, np.float32), np.zeros(2, np.int64)), E)
     assert (ky >> np.uint64(E.bit_length() - 1)) == (kx >> np.uint64(E.bit_length() - 1)) + np.uint64(1)
+
+
+def test_bc_swizzle_is_a_permutation_and_spreads_bank_groups():
+    """The M = 64 local search stores logical 16-byte chunk c of row r at
+    c ^ (r % 16) ^ (4 if c >= 8): a permutation of each row's 16 chunks; chunk
+    c of 4 consecutive rows and chunks c, c + 8 of one row (the two threads of
+    a row) land in distinct bank groups (a bank group: 4 banks = chunk mod 8)."""
+    def phys(r, c):
+        return (c ^ (r % 16) ^ (4 if c >= 8 else 0)) & 15
+
+    for r in range(64):
+        assert sorted(phys(r, c) for c in range(16)) == list(range(16))
+        for q in range(8):
+            assert phys(r, q) % 8 != phys(r, q + 8) % 8              # one row, both halves
+    for r0 in range(64):
+        for q in range(8):
+            rows = [(r0 + k) % 64 for k in range(4)]               # a quarter warp: 4 rows, 2 threads each
+            groups = [phys(r, q) % 8 for r in rows] + [phys(r, q + 8) % 8 for r in rows]
+            assert len(set(groups)) == 8
