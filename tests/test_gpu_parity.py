@@ -233,7 +233,8 @@ def test_mask_equals_rounding_of_exported_plan(c):
     assert torch.equal(m1, m2)
 
 
-@pytest.mark.parametrize("M,N,rows,cols", [(16, 8, 128, 128), (32, 16, 128, 256), (64, 32, 256, 512)])
+@pytest.mark.parametrize("M,N,rows,cols", [(4, 2, 64, 128), (8, 4, 64, 128), (16, 8, 128, 128), (32, 16, 128, 256),
+                                             (64, 32, 256, 512)])
 def test_rounding_bit_exact_on_adversarial_keys(M, N, rows, cols):
     """The bf16 sort's 32-bit keys keep a bucket of the plan (an exponent window
     and upper mantissa bits) and settle same-bucket runs with the full key: keys
