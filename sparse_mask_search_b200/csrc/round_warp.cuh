@@ -575,17 +575,28 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
                 // rows i and bp, and rows whose best partner was one of them, are
                 // rescanned: for M = 32 by the whole warp, one row at a time (a
                 // warp argmax over the row's cached gains: lowest partner on ties,
-                // the diagonal is -inf), for M = 16 each by its own lane (a row of
-                // 16 gains); every other row compares its best with its new
+                // the diagonal is -inf; rows i and bp from the new gains in the
+                // lanes' registers), for M = 16 each by its own lane (a row of 16
+                // gains); every other row compares its best with its new
                 // g(i, y), g(bp, y).  A/B: 16:32 3.499 -> 3.444 ms per call with
                 // the warp rescans, 8:16 1.125 -> 1.139 (so M = 16 keeps its own)
+                // A row whose best partner was i (bp) needs no rescan while its new
+                // gain with that partner has not fallen below the old best: every
+                // other partner's gain is unchanged and at most that value, and one
+                // equal to it has a higher index; the compare below then gives
+                // the same best as a rescan.  M = 16 rescans such rows anyway (its
+                // own-lane rescans are short: 8:16 1.067 -> 1.073 ms with the test,
+                // 16:32 3.286 -> 3.188 ms with it and the direct bests below).
                 const int op = row_thread ? sh.bestp[y] : 0;
-                const bool need = row_thread && (y == i || y == bp || op == i || op == bp);
+                const float ov = row_thread ? sh.bestv[y] : 0.f;
+                const bool mine = y == i || y == bp;
+                const bool fell = M < 32 || (op == i ? gi : gb) < ov;
+                const bool need = row_thread && (mine || ((op == i || op == bp) && fell));
                 if constexpr (M < 32) {
                     if (need) rescan_row<M>(sh, y);
                 }
                 if (row_thread && !need) {
-                    float bv = sh.bestv[y];
+                    float bv = ov;
                     int b2 = op;
                     const int c1 = i < bp ? i : bp, c2 = i < bp ? bp : i;
                     const float g1 = c1 == i ? gi : gb, g2 = c2 == i ? gi : gb;
@@ -594,7 +605,20 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
                     sh.bestv[y] = bv;
                     sh.bestp[y] = b2;
                 }
-                unsigned rows = M < 32 ? 0u : __ballot_sync(kFullMask, need);
+                if constexpr (M == 32) {
+                    // rows i and bp: their new gains are this warp's gi and gb (the
+                    // diagonal -inf; lane i's gb = g(bp, i) is lane bp's gi with
+                    // the two terms added in the other order, the same value)
+                    float vi = y == i ? -INFINITY : gi, vb = y == bp ? -INFINITY : gb;
+                    int pi = y, pb = y;
+                    warp_argmax(vi, pi);
+                    warp_argmax(vb, pb);
+                    if (lane == 0) {
+                        sh.bestv[i] = vi; sh.bestp[i] = pi;
+                        sh.bestv[bp] = vb; sh.bestp[bp] = pb;
+                    }
+                }
+                unsigned rows = M < 32 ? 0u : __ballot_sync(kFullMask, need && !mine);
                 while (rows) {
                     const int x = __ffs(static_cast<int>(rows)) - 1;
                     rows &= rows - 1;
@@ -1070,10 +1094,14 @@ __device__ void local_search_mp(const float* a, float* Bm, float* Cm, const Roun
                 // over the row's 64 cached gains, lowest partner on ties; the
                 // diagonal, which holds no gain, is skipped); every other row
                 // compares its best with its new g(i, y), g(bp, y)
+                // (a row whose best partner was i or bp and whose gain with it has
+                // not fallen keeps a best among i and bp, as in local_search)
                 const int op = sh.bestp[y];
-                const bool need = y == i || y == bp || op == i || op == bp;   // same for both threads of row y
+                const float ov = sh.bestv[y];
+                const bool need = y == i || y == bp ||
+                                  ((op == i || op == bp) && (op == i ? gi : gb) < ov);   // same for both threads of row y
                 if (!need && h == 0) {
-                    float bv = sh.bestv[y];
+                    float bv = ov;
                     int b2 = op;
                     const int c1 = i < bp ? i : bp, c2 = i < bp ? bp : i;
                     const float g1 = c1 == i ? gi : gb, g2 = c2 == i ? gi : gb;

@@ -300,3 +300,50 @@ def test_bc_swizzle_is_a_permutation_and_spreads_bank_groups():
             rows = [(r0 + k) % 64 for k in range(4)]               # a quarter warp: 4 rows, 2 threads each
             groups = [phys(r, q) % 8 for r in rows] + [phys(r, q + 8) % 8 for r in rows]
             assert len(set(groups)) == 8
+
+
+def test_best_partner_update_without_rescan_equals_rescan():
+    """After a swap of rows i and bp only the gains g(y, i), g(y, bp) of a row y
+    change.  The local search rescans row y only when its best partner was i or
+    bp AND its new gain with that partner fell below the old best; otherwise it
+    compares the old best with the two new gains (lowest partner on ties).  On
+    random tie-heavy gain tables that must equal a full rescan."""
+    rng = np.random.default_rng(3)
+
+    def rescan(G, y):
+        bv, bp = -np.inf, -1
+        for x in range(G.shape[0]):
+            if bp < 0 or G[y, x] > bv:
+                bv, bp = G[y, x], x
+        return bv, bp
+
+    checked = 0
+    for t in range(900):
+        M = (8, 16, 32)[t % 3]
+        lv = int(rng.integers(1, 5))
+        G = np.triu(rng.integers(-lv, lv + 1, (M, M)).astype(float), 1)
+        G = G + G.T
+        np.fill_diagonal(G, -np.inf)
+        old = [rescan(G, y) for y in range(M)]
+        i, bp = (int(v) for v in rng.choice(M, 2, replace=False))
+        for y in range(M):
+            if y != i:
+                G[i, y] = G[y, i] = float(rng.integers(-lv, lv + 1))
+        for y in range(M):
+            if y not in (i, bp):
+                G[bp, y] = G[y, bp] = float(rng.integers(-lv, lv + 1))
+        for y in range(M):
+            if y in (i, bp):
+                continue
+            ov, op = old[y]
+            gi, gb = G[y, i], G[y, bp]
+            if op in (i, bp) and (gi if op == i else gb) < ov:
+                continue                                       # rescanned
+            bv, b2 = ov, op
+            c1, c2 = min(i, bp), max(i, bp)
+            for c, g in ((c1, gi if c1 == i else gb), (c2, gi if c2 == i else gb)):
+                if g > bv or (g == bv and c < b2):
+                    bv, b2 = g, c
+            assert (bv, b2) == rescan(G, y)
+            checked += 1
+    assert checked > 10000
