@@ -295,6 +295,12 @@ __device__ bool greedy_and_repair(const float* a, const RoundView<M>& sh, int N,
         const int r0c = valid ? sh.rc[i] : N, c0c = valid ? sh.cc[j] : N;
         unsigned acc = 0u;
         unsigned und = __ballot_sync(kFullMask, valid && r0c < N && c0c < N);
+        {   // first pass: nothing accepted yet, so the lower bound rejects no lane
+            const bool mine = (und >> lane) & 1u;
+            const int ru = r0c + __popc(mr & lt & und), cu = c0c + __popc(mc & lt & und);
+            acc = __ballot_sync(kFullMask, mine && ru < N && cu < N);
+            und &= ~acc;
+        }
         while (und) {
             const bool mine = (und >> lane) & 1u;
             const unsigned maybe = acc | und;
