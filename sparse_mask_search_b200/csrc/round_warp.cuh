@@ -416,9 +416,10 @@ __device__ __forceinline__ float row_max(float t) {
 // partner: with N < M every row has a partner of finite gain (two rows with
 // the same support in every pair would put M ones in those columns); with
 // N = M every gain is -inf and no swap ever happens, whichever index is kept.
-// Quads are reduced independently, then merged in index order.
+// Quads are reduced independently, then merged in index order.  rescan_row_val
+// returns the best, rescan_row stores it in sh.bestv / sh.bestp.
 template <int M>
-__device__ __forceinline__ void rescan_row(const RoundView<M>& sh, int x) {
+__device__ __forceinline__ void rescan_row_val(const RoundView<M>& sh, int x, float& best_v, int& best_p) {
     constexpr int GS = M + 1;
     static_assert(M % 4 == 0, "quads");
     const float* row = sh.G + x * GS;
@@ -435,6 +436,14 @@ __device__ __forceinline__ void rescan_row(const RoundView<M>& sh, int x) {
         const int iq = s ? i23 : i01;
         if (q == 0 || vq > bv) { bv = vq; bp = iq; }
     }
+    best_v = bv;
+    best_p = bp;
+}
+template <int M>
+__device__ __forceinline__ void rescan_row(const RoundView<M>& sh, int x) {
+    float bv;
+    int bp;
+    rescan_row_val<M>(sh, x, bv, bp);
     sh.bestv[x] = bv;
     sh.bestp[x] = bp;
 }
@@ -472,7 +481,13 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
         }
     }
     ls_barrier<NT>();
-    if (row_thread && h == 0) rescan_row<M>(sh, y);
+    // each row's best partner and gain: M = 32 keeps them in the row's lane
+    // (reg_bests), M = 16 in shared memory
+    constexpr bool reg_bests = M == 32;
+    float my_bv = -INFINITY;
+    int my_bp = 0;
+    if constexpr (reg_bests) rescan_row_val<M>(sh, y, my_bv, my_bp);
+    else if (row_thread && h == 0) rescan_row<M>(sh, y);
 
     // The sweeps compute pair gains in max-plus form: with C_x[j] = a_xj off
     // row x's support (-inf on it) and Bn_x[j] = a_xj on it (+inf off it),
@@ -499,7 +514,7 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
     for (int sw = 0; sw < sweeps && quiet < M; ++sw) {
         for (int i = 0; i < M && quiet < M; ++i) {
             {   // skip anchors with no positive best gain (fixed between swaps)
-                const Bits P = __ballot_sync(kFullMask, lane < M && sh.bestv[lane] > 0.f);
+                const Bits P = __ballot_sync(kFullMask, lane < M && (reg_bests ? my_bv : sh.bestv[lane]) > 0.f);
                 const Bits ahead = P & (~Bits(0) << i);
                 if (!ahead) { quiet += M - i; break; }
                 const int nxt = lowest_bit(ahead);
@@ -507,8 +522,8 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
                 i = nxt;
                 if (quiet >= M) break;
             }
-            const float best = sh.bestv[i];
-            const int bp = sh.bestp[i];
+            const float best = reg_bests ? __shfl_sync(kFullMask, my_bv, i) : sh.bestv[i];
+            const int bp = reg_bests ? __shfl_sync(kFullMask, my_bp, i) : sh.bestp[i];
             if (!(best > 0.f)) { ++quiet; continue; }
             const Bits Oi = sh.rowbits[i], Ob = sh.rowbits[bp];
             // entries to exchange (every lane finds the same pair): lowest index on ties
@@ -526,11 +541,9 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
             quiet = 0;
             const Bits Oi2 = (Oi & ~(Bits(1) << j1)) | (Bits(1) << j2);
             const Bits Ob2 = (Ob & ~(Bits(1) << j2)) | (Bits(1) << j1);
-            ls_barrier<NT>();                        // everyone has read the old rows
-            if (tid == 0) {
-                sh.rowbits[i] = Oi2;
-                sh.rowbits[bp] = Ob2;
-            }
+            // sc was last read before the previous swap's final barrier, so it
+            // is written at once; the row masks after the next barrier, when
+            // every lane has read the old ones
             if (row_thread) {                        // rows i and bp after the swap: C, Bn, C, Bn
                 const bool ni = (Oi2 >> lane) & 1, nb = (Ob2 >> lane) & 1;
                 sh.sc[lane] = ni ? -INFINITY : ai;
@@ -539,6 +552,10 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
                 sh.sc[3 * M + lane] = nb ? ab : INFINITY;
             }
             ls_barrier<NT>();
+            if (tid == 0) {
+                sh.rowbits[i] = Oi2;
+                sh.rowbits[bp] = Ob2;
+            }
             if (y == i || y == bp) {                 // this lane's own row changed
                 const float* src = sh.sc + (y == i ? 0 : 2 * M);
 #pragma unroll
@@ -593,8 +610,8 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
                 // the same best as a rescan.  M = 16 rescans such rows anyway (its
                 // own-lane rescans are short: 8:16 1.067 -> 1.073 ms with the test,
                 // 16:32 3.286 -> 3.188 ms with it and the direct bests below).
-                const int op = row_thread ? sh.bestp[y] : 0;
-                const float ov = row_thread ? sh.bestv[y] : 0.f;
+                const int op = reg_bests ? my_bp : (row_thread ? sh.bestp[y] : 0);
+                const float ov = reg_bests ? my_bv : (row_thread ? sh.bestv[y] : 0.f);
                 const bool mine = y == i || y == bp;
                 const bool fell = M < 32 || (op == i ? gi : gb) < ov;
                 const bool need = row_thread && (mine || ((op == i || op == bp) && fell));
@@ -608,8 +625,13 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
                     const float g1 = c1 == i ? gi : gb, g2 = c2 == i ? gi : gb;
                     if (g1 > bv || (g1 == bv && c1 < b2)) { bv = g1; b2 = c1; }
                     if (g2 > bv || (g2 == bv && c2 < b2)) { bv = g2; b2 = c2; }
-                    sh.bestv[y] = bv;
-                    sh.bestp[y] = b2;
+                    if constexpr (reg_bests) {
+                        my_bv = bv;
+                        my_bp = b2;
+                    } else {
+                        sh.bestv[y] = bv;
+                        sh.bestp[y] = b2;
+                    }
                 }
                 if constexpr (M == 32) {
                     // rows i and bp: their new gains are this warp's gi and gb (the
@@ -619,10 +641,8 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
                     int pi = y, pb = y;
                     warp_argmax(vi, pi);
                     warp_argmax(vb, pb);
-                    if (lane == 0) {
-                        sh.bestv[i] = vi; sh.bestp[i] = pi;
-                        sh.bestv[bp] = vb; sh.bestp[bp] = pb;
-                    }
+                    if (lane == i) { my_bv = vi; my_bp = pi; }
+                    if (lane == bp) { my_bv = vb; my_bp = pb; }
                 }
                 unsigned rows = M < 32 ? 0u : __ballot_sync(kFullMask, need && !mine);
                 while (rows) {
@@ -631,9 +651,9 @@ __device__ void local_search(const float* a, const RoundView<M>& sh, int sweeps,
                     float g = lane < M ? sh.G[x * GS + lane] : -INFINITY;
                     int p = lane;
                     warp_argmax(g, p);
-                    if (lane == 0) {
-                        sh.bestv[x] = g;
-                        sh.bestp[x] = p;
+                    if (lane == x) {                    // M = 32: reg_bests
+                        my_bv = g;
+                        my_bp = p;
                     }
                 }
             }
