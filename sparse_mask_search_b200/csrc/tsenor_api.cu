@@ -3,6 +3,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <new>
 #include <type_traits>
 
 #include <cudaTypedefs.h>
@@ -342,6 +343,30 @@ extern "C" tsenor_status tsenor_plan_warm(const void* W, tsenor_dtype dtype, int
 }
 
 // ---------------------------------------------------------------------------
+// The context current on the calling thread (driver entry point fetched once
+// through the runtime): resources cached across calls are keyed by it, so a
+// new primary context after cudaDeviceReset gets fresh ones.  *ctx is null
+// while the runtime has not yet made a context current on this thread.
+namespace {
+constexpr int kMaxDevices = 64;
+PFN_cuCtxGetCurrent g_ctx_current = nullptr;
+std::once_flag g_ctx_once;
+
+cudaError_t current_context(CUcontext* ctx) {
+    std::call_once(g_ctx_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent>(fn);
+    });
+    if (!g_ctx_current) return cudaErrorNotSupported;
+    *ctx = nullptr;
+    return g_ctx_current(ctx) == CUDA_SUCCESS ? cudaSuccess : cudaErrorDeviceUninitialized;
+}
+}  // namespace
+
+// ---------------------------------------------------------------------------
 // tsenor_mask_host: row chunks of a host matrix pipelined through two device
 // slots.  Copies run on an internal stream X, solves alternate between the
 // caller's stream and a second internal stream (so that one chunk's tail
@@ -352,29 +377,70 @@ extern "C" tsenor_status tsenor_plan_warm(const void* W, tsenor_dtype dtype, int
 //      into dW[s] (free: chunk k's solve is done); event h2d[k+2]
 // so each upload overlaps the solve of the chunk before it.  The caller's
 // stream then waits for X's last copy.
+// The two internal streams and the events are created on a host thread's
+// first call on a device (and context) and kept for its later calls:
+// creating and destroying them took most of a call's host time, and the
+// first upload waited for it (the 16:32 workload's call spent about 0.5 ms
+// on the host before).  An event is recorded once per call, and every wait
+// on it is enqueued in the same call, after that record, so reuse across
+// calls is safe; calls of one thread share the streams and so run in order.
+// They are never destroyed: they go with the context.
 namespace {
 constexpr int kHostMaxChunks = 64;
+constexpr int kHostEvents = 2 * kHostMaxChunks + 2;
+
+struct HostPipeRes {
+    CUcontext ctx = nullptr;
+    cudaStream_t x = nullptr, c2 = nullptr;
+    cudaEvent_t ev[kHostEvents] = {};
+};
+thread_local HostPipeRes* tl_pipe[kMaxDevices];   // allocated on first use, never freed
+
+// This thread's streams and events on the current device and context.
+cudaError_t host_pipe_res(HostPipeRes** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    CUcontext ctx = nullptr;
+    e = current_context(&ctx);
+    if (e != cudaSuccess) return e;
+    if (!tl_pipe[dev]) tl_pipe[dev] = new (std::nothrow) HostPipeRes();
+    if (!tl_pipe[dev]) return cudaErrorMemoryAllocation;
+    HostPipeRes& r = *tl_pipe[dev];
+    if (!r.x || !ctx || r.ctx != ctx) {
+        HostPipeRes fresh;                           // a stale context's handles are dropped, not destroyed
+        e = cudaStreamCreateWithFlags(&fresh.x, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&fresh.c2, cudaStreamNonBlocking);
+        for (int i = 0; i < kHostEvents && e == cudaSuccess; ++i)
+            e = cudaEventCreateWithFlags(&fresh.ev[i], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = current_context(&fresh.ctx);
+        if (e == cudaSuccess && !fresh.ctx) e = cudaErrorDeviceUninitialized;
+        if (e != cudaSuccess) {
+            for (int i = 0; i < kHostEvents; ++i)
+                if (fresh.ev[i]) cudaEventDestroy(fresh.ev[i]);
+            if (fresh.x) cudaStreamDestroy(fresh.x);
+            if (fresh.c2) cudaStreamDestroy(fresh.c2);
+            return e;
+        }
+        r = fresh;
+    }
+    *out = &r;
+    return cudaSuccess;
+}
 
 struct HostPipe {
     cudaStream_t x = nullptr, c2 = nullptr;
-    cudaEvent_t ev[2 * kHostMaxChunks + 2] = {};
+    cudaEvent_t* ev = nullptr;
     int nev = 0;
     void* dW[2] = {nullptr, nullptr};
     uint32_t* dm[2] = {nullptr, nullptr};
-    cudaEvent_t event() {
-        cudaEvent_t e = nullptr;
-        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
-        ev[nev++] = e;
-        return e;
-    }
+    cudaEvent_t event() { return nev < kHostEvents ? ev[nev++] : nullptr; }
     void release(cudaStream_t st) {
         for (int s = 0; s < 2; ++s) {
             if (dW[s]) cudaFreeAsync(dW[s], st);
             if (dm[s]) cudaFreeAsync(dm[s], st);
         }
-        for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
-        if (x) cudaStreamDestroy(x);
-        if (c2) cudaStreamDestroy(c2);
     }
 };
 }  // namespace
@@ -400,8 +466,12 @@ extern "C" tsenor_status tsenor_mask_host(const void* W_host, tsenor_dtype dtype
     const int64_t nchunks = (rows + chunk - 1) / chunk;
 
     HostPipe p;
-    cudaError_t e = cudaStreamCreateWithFlags(&p.x, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p.c2, cudaStreamNonBlocking);
+    HostPipeRes* res = nullptr;
+    cudaError_t e = host_pipe_res(&res);
+    if (e != cudaSuccess) return cuda_fail(e, "tsenor_mask_host streams");
+    p.x = res->x;
+    p.c2 = res->c2;
+    p.ev = res->ev;
     for (int s = 0; s < 2 && e == cudaSuccess; ++s) {
         e = cudaMallocAsync(&p.dW[s], size_t(chunk) * size_t(cols) * es, st);
         if (e == cudaSuccess)
@@ -561,12 +631,9 @@ extern "C" const char* tsenor_last_error(void) { return tsenor::g_last_error; }
 static __device__ __align__(256) float g_noalloc_plan[TSENOR_NOALLOC_MAX_PARAMS];
 
 namespace {
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 float* g_noalloc_ptr[kMaxDevices] = {};
 CUcontext g_noalloc_ctx[kMaxDevices] = {};
-PFN_cuCtxGetCurrent g_ctx_current = nullptr;
-std::once_flag g_ctx_once;
 
 // Device address of g_noalloc_plan on the current device and context.
 cudaError_t noalloc_plan_ptr(float** out) {
@@ -574,24 +641,19 @@ cudaError_t noalloc_plan_ptr(float** out) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::call_once(g_ctx_once, [] {
-        void* fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent>(fn);
-    });
-    if (!g_ctx_current) return cudaErrorNotSupported;
     // no current context yet on this thread (the runtime makes the primary
     // context current lazily): the symbol lookup below does that first
     CUcontext ctx = nullptr;
-    if (g_ctx_current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+    e = current_context(&ctx);
+    if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
     if (!g_noalloc_ptr[dev] || !ctx || g_noalloc_ctx[dev] != ctx) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_plan);
         if (e != cudaSuccess) return e;
-        if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
+        e = current_context(&ctx);
+        if (e != cudaSuccess) return e;
+        if (!ctx) return cudaErrorDeviceUninitialized;
         g_noalloc_ptr[dev] = static_cast<float*>(p);
         g_noalloc_ctx[dev] = ctx;
     }
