@@ -120,6 +120,40 @@ def test_host_pipeline_matches_device_call(rows, cols, M, N, dtype):
     assert torch.equal(out2, ref)
 
 
+def test_host_pipeline_from_two_threads():
+    """Each host thread keeps its own pipeline streams and events: two threads
+    calling tsenor_mask_host at the same time, several times each on their own
+    streams, all get tsenor_mask's mask."""
+    import threading
+    stor, W = synth.make_matrix(4096, 2048, "bf16", "t3_outlier_cols", 0.02, seed=11)
+    Wd = to_device(stor, "bf16")
+    ref = tsl.tsenor_mask(Wd, 16, 32, 20.0, 120, 4).cpu()
+    Wh = Wd.cpu().pin_memory()
+    outs, errs = [None, None], []
+
+    def run(k):
+        try:
+            torch.cuda.set_device(Wd.device)
+            s = torch.cuda.Stream()
+            got = []
+            for _ in range(3):
+                got.append(tsl.tsenor_mask_host(Wh, 16, 32, 20.0, 120, 4, stream=s))
+            s.synchronize()
+            outs[k] = got
+        except Exception as e:                      # reported below, in the main thread
+            errs.append(e)
+
+    threads = [threading.Thread(target=run, args=(k,)) for k in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errs, errs
+    for got in outs:
+        for o in got:
+            assert torch.equal(o, ref)
+
+
 @pytest.mark.parametrize("M,N", [(8, 4), (16, 8), (32, 16), (64, 32)])
 def test_offsets_beyond_int32(M, N):
     """A matrix of more than 2^31 elements (bf16, generated on the device from a
