@@ -245,8 +245,9 @@ tsenor_status tsenor_mask_scores(const float* scores, int64_t rows, int64_t cols
  * Uses stream-ordered device workspaces for two W chunks and two mask chunks
  * (cudaMallocAsync / cudaFreeAsync).  The two internal streams and their
  * events are created on a host thread's first call on a device (and context)
- * and reused by that thread's later calls, which therefore run one after the
- * other on the device; they are never destroyed (they go with the context).  Errors as tsenor_mask; TSENOR_ERR_ARG
+ * and reused by that thread's later calls (whose copies therefore queue
+ * behind the earlier calls' copies); they are never destroyed (they go with
+ * the context).  Errors as tsenor_mask; TSENOR_ERR_ARG
  * also for a null host pointer.  The review has no counterpart of this call.
  */
 tsenor_status tsenor_mask_host(const void* W_host, tsenor_dtype dtype, int64_t rows, int64_t cols, int N, int M,
